@@ -1,0 +1,282 @@
+/*
+ * Oracle for the routed mixture-of-experts layer -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow CPU restatement of what the layer computes, in fp64, written
+ * from the pages' description and sharing no code with the CUDA library.  Only
+ * the tests, the package smoke check and the benchmark's CPU-baseline leg may
+ * load it.  Every quantity is converted exactly to double (bf16 -> its value,
+ * int8 -> q*s, int4 -> q*s) and accumulated in fp64 in index order; there is no
+ * blocking, fusion or reordering beyond the definition.
+ *
+ * The layer, per token t (sources named per step below):
+ *   1. logits   l_e = sum_h W_r[e,h] x[t,h]                   for every expert e
+ *   2. keys     sigmoid router: s_e = 1/(1+exp(-l_e)), key_e = s_e + b_e
+ *               softmax router: key_e = exp(l_e - m) / sum_{a active} exp(l_a - m)
+ *      "sigmoid scores, the top 8 chosen on the scores plus the correction
+ *       bias, weights renormalized and scaled by 2.446" -- Kimi-Linear LiteRT-LM
+ *       details page, Conversion notes, mixture-of-experts bullet; "the sigmoid
+ *       MoE router with its selection bias" -- CMF code specialist page, How it
+ *       was made step 1.  "The router, its softmax, the top 8 and their
+ *       renormalization are ordinary ops" -- Qwen3-30B-A3B LiteRT-LM card,
+ *       Conversion Notes.
+ *   3. top-k    sort the ACTIVE experts by (key descending, index ascending) and
+ *               keep the first k; masked experts are never selectable ("Runtime
+ *               semantics equal the runtime expert mask" -- CMF page, Defrag).
+ *   4. weights  w_j = r_j / sum_{selected} r * scale, with r = s (sigmoid scores,
+ *               WITHOUT the bias, which only selects) or r = p (softmax).
+ *   5. experts  for each selected e: g = W_gate[e] x, u = W_up[e] x,
+ *               a = g * sigmoid(g) * u  (SiLU-gated), o = W_down[e] a.
+ *               "only the 8 routed experts are computed for each token" --
+ *               Qwen3 card, Conversion Notes; activation 'silu' -- same card and
+ *               the Kimi details page (moe op with SiLU).
+ *   6. combine  y[t] = sum_j w_j o_j in slot order; no residual add (the add
+ *               sits outside the moe op -- Qwen3 card, Conversion Notes,
+ *               moe_fusion_guard bullet).
+ *
+ * Stored formats read here (rows are output channels, columns the reduction):
+ *   W_gate, W_up [E, I, H]; W_down [E, H, I]
+ *   f32 / bf16 (raw 16-bit patterns) / int8 with s[E, rows] (one scale per
+ *   output row and expert -- Kimi details page, quantization bullet) / int4
+ *   packed two per byte, low nibble = even column, two's complement, with
+ *   s[E, rows, cols/32] (block 32, fp32 scales -- Qwen3 card, Artifacts table).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_INT8 = 2, ORC_INT4 = 3 };
+enum { ORC_SIGMOID = 0, ORC_SOFTMAX = 1 };
+enum { ORC_GATE = 0, ORC_UP = 1, ORC_DOWN = 2 };
+
+typedef struct {
+  int32_t H, I, E, k;
+  int32_t router; /* ORC_SIGMOID or ORC_SOFTMAX */
+  int32_t wfmt;   /* expert storage format */
+  int32_t xfmt;   /* ORC_F32 or ORC_BF16 */
+  int32_t pad;
+  double scale;   /* 2.446 (Kimi) or 1 (Qwen3) */
+  const float* W_r;      /* [E, H] */
+  const float* b;        /* [E] or NULL (= zero bias) */
+  const uint8_t* mask;   /* [E] 1 = active, or NULL (all active) */
+  const void* W_gate;
+  const void* W_up;
+  const void* W_down;
+  const float* s_gate;
+  const float* s_up;
+  const float* s_down;
+} oracle_layer;
+
+/* ---------------------------------------------------------------- decoding */
+
+static double bf16_value(uint16_t bits) {
+  uint32_t u = (uint32_t)bits << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+static double x_value(const oracle_layer* L, const void* x, int64_t t, int64_t h) {
+  if (L->xfmt == ORC_BF16) return bf16_value(((const uint16_t*)x)[t * L->H + h]);
+  return (double)((const float*)x)[t * L->H + h];
+}
+
+/* value of expert weight (row, col) of matrix `which` of expert e */
+double oracle_weight(const oracle_layer* L, int which, int64_t e, int64_t row, int64_t col) {
+  const int64_t R = (which == ORC_DOWN) ? L->H : L->I;
+  const int64_t C = (which == ORC_DOWN) ? L->I : L->H;
+  const void* W = which == ORC_GATE ? L->W_gate : which == ORC_UP ? L->W_up : L->W_down;
+  const float* S = which == ORC_GATE ? L->s_gate : which == ORC_UP ? L->s_up : L->s_down;
+  const int64_t r = e * R + row;
+  switch (L->wfmt) {
+    case ORC_F32:
+      return (double)((const float*)W)[r * C + col];
+    case ORC_BF16:
+      return bf16_value(((const uint16_t*)W)[r * C + col]);
+    case ORC_INT8:
+      return (double)((const int8_t*)W)[r * C + col] * (double)S[r];
+    case ORC_INT4: {
+      const uint8_t byte = ((const uint8_t*)W)[r * (C / 2) + col / 2];
+      int nib = (col & 1) ? (byte >> 4) : (byte & 0xF);
+      if (nib >= 8) nib -= 16;
+      return (double)nib * (double)S[r * (C / 32) + col / 32];
+    }
+  }
+  return NAN;
+}
+
+static int is_active(const oracle_layer* L, int e) { return L->mask == NULL || L->mask[e] != 0; }
+
+static int count_active(const oracle_layer* L) {
+  int n = 0;
+  for (int e = 0; e < L->E; ++e) n += is_active(L, e);
+  return n;
+}
+
+static double sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }
+
+/* ------------------------------------------------------------------ router */
+
+/* logits[(t - t0) * E + e] for tokens [t0, t1), all experts (masking is a selection rule) */
+int oracle_router_logits(const oracle_layer* L, const void* x, int64_t t0, int64_t t1, double* logits) {
+  if (!L || !x || !logits || t1 < t0) return -1;
+  for (int64_t t = t0; t < t1; ++t)
+    for (int64_t e = 0; e < L->E; ++e) {
+      double acc = 0.0;
+      for (int64_t h = 0; h < L->H; ++h) acc += (double)L->W_r[e * L->H + h] * x_value(L, x, t, h);
+      logits[(t - t0) * L->E + e] = acc;
+    }
+  return 0;
+}
+
+typedef struct {
+  double key;
+  int e;
+} ranked;
+
+/* key descending, then expert index ascending */
+static int by_key_then_index(const void* pa, const void* pb) {
+  const ranked* a = (const ranked*)pa;
+  const ranked* b = (const ranked*)pb;
+  if (a->key > b->key) return -1;
+  if (a->key < b->key) return 1;
+  return a->e < b->e ? -1 : (a->e > b->e ? 1 : 0);
+}
+
+/* selection keys of every expert for one token (masked experts get -inf) */
+int oracle_keys(const oracle_layer* L, const double* logits, double* keys) {
+  if (!L || !logits || !keys) return -1;
+  if (L->router == ORC_SIGMOID) {
+    for (int e = 0; e < L->E; ++e)
+      keys[e] = is_active(L, e) ? sigmoid(logits[e]) + (L->b ? (double)L->b[e] : 0.0) : -INFINITY;
+    return 0;
+  }
+  if (L->router == ORC_SOFTMAX) {
+    double m = -INFINITY, z = 0.0;
+    for (int e = 0; e < L->E; ++e)
+      if (is_active(L, e) && logits[e] > m) m = logits[e];
+    for (int e = 0; e < L->E; ++e)
+      if (is_active(L, e)) z += exp(logits[e] - m);
+    for (int e = 0; e < L->E; ++e) keys[e] = is_active(L, e) ? exp(logits[e] - m) / z : -INFINITY;
+    return 0;
+  }
+  return -1;
+}
+
+/*
+ * Route one token from its logits: idx[k], w[k] in descending key order, and
+ * margin = key of the k-th selected minus key of the best unselected active
+ * expert (+inf when every active expert is selected).
+ */
+int oracle_select(const oracle_layer* L, const double* logits, int32_t* idx, double* w, double* margin) {
+  const int E = L->E, k = L->k;
+  const int n_act = count_active(L);
+  if (k < 1 || k > n_act) return -1;
+  double* keys = (double*)malloc(sizeof(double) * E);
+  ranked* order = (ranked*)malloc(sizeof(ranked) * n_act);
+  if (!keys || !order || oracle_keys(L, logits, keys) != 0) {
+    free(keys);
+    free(order);
+    return -1;
+  }
+  int n = 0;
+  for (int e = 0; e < E; ++e)
+    if (is_active(L, e)) {
+      order[n].key = keys[e];
+      order[n].e = e;
+      ++n;
+    }
+  qsort(order, n, sizeof(ranked), by_key_then_index);
+  double total = 0.0;
+  for (int j = 0; j < k; ++j) {
+    const int e = order[j].e;
+    const double r = (L->router == ORC_SIGMOID) ? sigmoid(logits[e]) : keys[e];
+    idx[j] = e;
+    w[j] = r;
+    total += r;
+  }
+  for (int j = 0; j < k; ++j) w[j] = w[j] / total * L->scale;
+  if (margin) *margin = (k < n) ? order[k - 1].key - order[k].key : INFINITY;
+  free(keys);
+  free(order);
+  return 0;
+}
+
+/* route tokens [t0, t1): idx/w/margin are indexed by (t - t0) */
+int oracle_route(const oracle_layer* L, const void* x, int64_t t0, int64_t t1, int32_t* idx, double* w,
+                 double* margin) {
+  if (!L || !x || !idx || !w || t1 < t0) return -1;
+  double* logits = (double*)malloc(sizeof(double) * L->E);
+  if (!logits) return -1;
+  int rc = 0;
+  for (int64_t t = t0; t < t1 && rc == 0; ++t) {
+    rc = oracle_router_logits(L, x, t, t + 1, logits);
+    if (rc == 0)
+      rc = oracle_select(L, logits, idx + (t - t0) * L->k, w + (t - t0) * L->k, margin ? margin + (t - t0) : NULL);
+  }
+  free(logits);
+  return rc;
+}
+
+/* ----------------------------------------------------------------- experts */
+
+/* o[H] = W_down[e] (SiLU(W_gate[e] xt) * (W_up[e] xt)) for one token vector xt[H] */
+int oracle_expert(const oracle_layer* L, int64_t e, const double* xt, double* o) {
+  if (!L || !xt || !o || e < 0 || e >= L->E) return -1;
+  const int64_t H = L->H, I = L->I;
+  double* a = (double*)malloc(sizeof(double) * I);
+  if (!a) return -1;
+  for (int64_t i = 0; i < I; ++i) {
+    double g = 0.0, u = 0.0;
+    for (int64_t h = 0; h < H; ++h) {
+      g += oracle_weight(L, ORC_GATE, e, i, h) * xt[h];
+      u += oracle_weight(L, ORC_UP, e, i, h) * xt[h];
+    }
+    a[i] = g * sigmoid(g) * u;
+  }
+  for (int64_t r = 0; r < H; ++r) {
+    double acc = 0.0;
+    for (int64_t i = 0; i < I; ++i) acc += oracle_weight(L, ORC_DOWN, e, r, i) * a[i];
+    o[r] = acc;
+  }
+  free(a);
+  return 0;
+}
+
+/*
+ * y for tokens [t0, t1) under a GIVEN routing: y[(t - t0) * H + h] =
+ * sum_j w[j] o_{idx[j]}[h] in slot order.  idx/w are indexed by (t - t0).
+ */
+int oracle_combine(const oracle_layer* L, const void* x, int64_t t0, int64_t t1, const int32_t* idx,
+                   const double* w, double* y) {
+  if (!L || !x || !idx || !w || !y || t1 < t0) return -1;
+  const int64_t H = L->H;
+  double* xt = (double*)malloc(sizeof(double) * H);
+  double* o = (double*)malloc(sizeof(double) * H);
+  if (!xt || !o) {
+    free(xt);
+    free(o);
+    return -1;
+  }
+  int rc = 0;
+  for (int64_t t = t0; t < t1 && rc == 0; ++t) {
+    for (int64_t h = 0; h < H; ++h) xt[h] = x_value(L, x, t, h);
+    double* yt = y + (t - t0) * H;
+    for (int64_t h = 0; h < H; ++h) yt[h] = 0.0;
+    for (int j = 0; j < L->k && rc == 0; ++j) {
+      rc = oracle_expert(L, idx[(t - t0) * L->k + j], xt, o);
+      for (int64_t h = 0; h < H; ++h) yt[h] += w[(t - t0) * L->k + j] * o[h];
+    }
+  }
+  free(xt);
+  free(o);
+  return rc;
+}
+
+/* the whole layer for tokens [t0, t1): route, then combine under that routing */
+int oracle_forward(const oracle_layer* L, const void* x, int64_t t0, int64_t t1, int32_t* idx, double* w,
+                   double* margin, double* y) {
+  int rc = oracle_route(L, x, t0, t1, idx, w, margin);
+  if (rc == 0) rc = oracle_combine(L, x, t0, t1, idx, w, y);
+  return rc;
+}
