@@ -1,0 +1,437 @@
+"""Benchmark of the routed mixture-of-experts layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl {ours,reference}]
+
+One step = one pass of the whole layer (router -> expert-sorted order ->
+gate/up -> down -> combine) over one batch of the workload, through the C ABI
+(moe_route + moe_forward).  Default workload: the Kimi-shaped decode batch
+(T=32, H=2304, E=256, k=8, I=2048, bf16 weights).
+
+  value  tokens/s over the timed steps, inputs resident in HBM; each step timed
+         with CUDA events on the launching stream, L2 flushed (a 512 MB write)
+         between steps outside the timed intervals.
+  e2e    the same metric with x copied host->device from pinned memory and y
+         copied back inside each timed step.
+  roofline  the dominant kernel's algorithmic bytes (or flops) per launch over
+         its event-timed average duration, against MEASURED_PEAKS.json.
+  cpu_baseline  the fp64 oracle on the host cores over a bounded token sample.
+
+Multi-GPU: the layer does not shard on one node's hot path (one GPU, no
+sharding), so --gpus N runs N independent replicas, one per rank, each on its
+own batch ("scaling": "weak"); torch.distributed carries only the barrier and
+the max-over-ranks of the timed duration.
+
+--impl reference runs the reference arm: the fp64 oracle (the only reference
+implementation there is) timed on the host cores, on the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "routed-MoE layer tokens/s at 1 B200"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DOMINANT = {  # kernel whose roofline is reported, per path
+    "gemv": "gemv_gateup",
+    "gemm": "gemm_gateup",
+}
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def dist_init(backend: str):
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def max_over_ranks(v: float, device=None) -> float:
+    """Max of a float over all ranks (the timed duration of the slowest replica)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(v)
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- clocks
+
+CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    """nvidia-smi sampling every 200 ms while the timed region runs."""
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", "moe_bench_clocks_%d_%d.csv" % (os.getpid(), gpu_index))
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + CLOCK_QUERY,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [c.strip() for c in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": sorted(reasons)}
+        busy = [s for s in sm if smax and s >= 0.3 * smax] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- workload accounting
+
+def touched_experts(idx: np.ndarray, E: int) -> int:
+    return int(np.unique(idx[(idx >= 0) & (idx < E)]).size)
+
+
+def algorithmic(prob, idx: np.ndarray):
+    """Per-launch algorithmic bytes / flops of the kernels, and the layer totals.
+
+    gate/up: per touched expert, the gate and up weight (+scale) bytes; plus x
+    read and h written.  down: per touched expert its down weight (+scale)
+    bytes; plus h read and the per-pair outputs written.  Flops count only the
+    routed work: 6*H*I per (token, slot) pair and 2*H*E for the router.
+    """
+    E, H, I, T, k = prob.E, prob.H, prob.I, prob.T, prob.k
+    ut = touched_experts(idx, E)
+    P = T * k
+    xb = 2 if prob.xfmt == "bf16" else 4
+    hb = 4 if prob.wfmt == "f32" else 2
+    per_mat = lambda W, S: W.nbytes // E + (0 if S is None else S.nbytes // E)
+    gate_up_per_expert = per_mat(prob.W_gate, prob.s_gate) + per_mat(prob.W_up, prob.s_up)
+    down_per_expert = per_mat(prob.W_down, prob.s_down)
+    bytes_ = {
+        "gemv_gateup": ut * gate_up_per_expert + T * H * xb + P * I * hb,
+        "gemm_gateup": ut * gate_up_per_expert + P * H * 2 + P * I * 2,
+        "gemv_down": ut * down_per_expert + P * I * hb + P * H * 4,
+        "gemm_down": ut * down_per_expert + P * I * 2 + P * H * 4,
+    }
+    flops = {"gemm_gateup": 4.0 * P * H * I, "gemm_down": 2.0 * P * H * I, "gemv_gateup": 4.0 * P * H * I,
+             "gemv_down": 2.0 * P * H * I}
+    layer_bytes = ut * (gate_up_per_expert + down_per_expert) + prob.W_r.nbytes + 2 * T * H * xb
+    layer_flops = 6.0 * P * H * I + 2.0 * T * H * E
+    return dict(touched=ut, per_expert_gate_up=gate_up_per_expert, per_expert_down=down_per_expert, bytes=bytes_,
+                flops=flops, layer_bytes=layer_bytes, layer_flops=layer_flops)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        try:
+            d = json.load(open(p))
+            return d, "measured"
+        except (OSError, ValueError):
+            pass
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def known_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+    except (OSError, ValueError):
+        return None
+    ent = d.get(kernel, {}).get(workload)
+    if not ent:
+        return None
+    src = os.path.join(ROOT, ent["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != ent["source_sha256"]:
+        return None
+    return ent["dram_bytes_per_launch"]
+
+
+# ----------------------------------------------------------------------------- CPU oracle timing
+
+def cpu_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def time_oracle(prob, budget_s: float, max_tokens=None):
+    """Time the fp64 oracle (route + experts + combine) on a seeded token sample
+    sized to roughly `budget_s` seconds of work; returns (tokens/s, threads, sample text)."""
+    import oracle
+    cores = cpu_threads()
+    orc = oracle.Oracle(prob, nthreads=cores)
+    t0 = time.perf_counter()
+    orc.forward([0])
+    per_token = max(time.perf_counter() - t0, 1e-6)  # one token, one thread
+    n = int(budget_s * cores / per_token)
+    n = max(1, min(n, prob.T if max_tokens is None else min(prob.T, max_tokens)))
+    rng = np.random.default_rng(0)
+    toks = np.sort(rng.choice(prob.T, n, replace=False))
+    t0 = time.perf_counter()
+    orc.forward(toks)
+    dt = time.perf_counter() - t0
+    return n / dt, cores, "%d of %d tokens (seeded), route + experts + combine in fp64" % (n, prob.T)
+
+
+# ----------------------------------------------------------------------------- arms
+
+def config_block(prob, cid, extra=None):
+    c = {"workload": prob.cfg["workload"], "T": prob.T, "H": prob.H, "E": prob.E, "k": prob.k, "I": prob.I,
+         "experts": prob.wfmt, "activations": prob.xfmt, "router": prob.router,
+         "active_experts": int(prob.mask.sum()) if prob.mask is not None else prob.E,
+         "l2": "flushed between steps (512 MB write, outside timed intervals); expert weights >> L2",
+         "parallelism": "replicas"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+def run_reference(args):
+    rank, world = dist_init("gloo")
+    if rank != 0:
+        return 0
+    prob = synth.make_problem(args.config)
+    import oracle
+    cores = cpu_threads()
+    orc = oracle.Oracle(prob, nthreads=cores)
+    t0 = time.perf_counter()
+    orc.forward([0])
+    per_token = max(time.perf_counter() - t0, 1e-6)
+    # each step: a token sample worth about 6 s of oracle work on all cores
+    n = max(1, min(prob.T, int(6.0 * cores / per_token)))
+    rng = np.random.default_rng(1)
+    times = []
+    for step in range(args.warmup + args.steps):
+        toks = np.sort(rng.choice(prob.T, n, replace=False))
+        t0 = time.perf_counter()
+        orc.forward(toks)
+        dt = time.perf_counter() - t0
+        if step >= args.warmup:
+            times.append(dt)
+    sec = sum(times) / len(times)
+    value = n / sec
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_block(prob, args.config, {"sample_tokens_per_step": n}),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": "%d of %d tokens per step (seeded), route + experts + combine in fp64"
+                                       % (n, prob.T)},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dist_init("nccl")
+    import mixture_experts_layer_31_b200 as moe
+    dev = torch.device("cuda", local)
+    prob = synth.make_problem(args.config)
+    path = {"auto": moe.MOE_PATH_AUTO, "gemv": moe.MOE_PATH_GEMV, "gemm": moe.MOE_PATH_GEMM}[args.path]
+    layer = moe.MoELayer(H=prob.H, I=prob.I, E=prob.E, k=prob.k, router=prob.router, scale=prob.scale,
+                         wfmt=prob.wfmt, xfmt=prob.xfmt, W_r=prob.W_r, b=prob.b, expert_mask=prob.mask,
+                         W_gate=prob.W_gate, W_up=prob.W_up, W_down=prob.W_down, s_gate=prob.s_gate,
+                         s_up=prob.s_up, s_down=prob.s_down, path=path, device=dev)
+    if prob.xfmt == "bf16":
+        x_host = torch.from_numpy(prob.x.view(np.int16)).view(torch.bfloat16)
+    else:
+        x_host = torch.from_numpy(prob.x)
+    x = x_host.to(dev)
+    T, k = prob.T, prob.k
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    y = torch.empty((T, prob.H), dtype=layer.x_dtype, device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(xin, yout):
+        layer.route(xin, out=(idx, w))
+        layer.forward(xin, idx, w, y=yout)
+
+    for _ in range(max(args.warmup, 3) if args.warmup > 0 else 0):
+        step(x, y)
+    torch.cuda.synchronize(dev)
+    idx_np = idx.cpu().numpy()
+    acc = algorithmic(prob, idx_np)
+
+    # ---- device-resident timed region (per-kernel events on for the roofline)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    moe.moe_stage_times()
+    moe.moe_stage_timing(True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    n0 = moe.moe_launch_count()
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step(x, y)
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+    launches = moe.moe_launch_count() - n0
+    moe.moe_stage_timing(False)
+    stages = moe.moe_stage_times()
+    step_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
+    step_ms = max_over_ranks(step_ms, dev)
+    value = world * T / (step_ms * 1e-3)
+
+    # ---- end to end: pinned host x in, pinned host y out, copies inside each timed step
+    xh = x_host.pin_memory()
+    yh = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    xd = torch.empty_like(x)
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for _ in range(2):
+        xd.copy_(xh, non_blocking=True)
+        step(xd, y)
+        yh.copy_(y, non_blocking=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        e_starts[i].record(stream)
+        xd.copy_(xh, non_blocking=True)
+        step(xd, y)
+        yh.copy_(y, non_blocking=True)
+        e_ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)) / args.steps, dev)
+
+    # ---- roofline of the dominant kernel
+    peaks, peak_src = load_peaks()
+    path_used = "gemm" if "gemm_gateup" in stages else "gemv"
+    kern = DOMINANT[path_used]
+    launches_k, total_k = stages.get(kern, (0, 0.0))
+    avg_ms = total_k / max(launches_k, 1)
+    if path_used == "gemv":
+        achieved = acc["bytes"][kern] / (avg_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "kernel": kern, "avg_launch_ms": avg_ms,
+                "algorithmic_bytes_per_launch": acc["bytes"][kern],
+                "peak_source": "%s hbm_gbs (%s)" % ("MEASURED_PEAKS.json" if peak_src == "measured" else "fallback",
+                                                    "of measured" if peak_src == "measured" else "of fallback")}
+    else:
+        achieved = acc["flops"][kern] / (avg_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "kernel": kern, "avg_launch_ms": avg_ms,
+                "algorithmic_flops_per_launch": acc["flops"][kern],
+                "peak_source": "bf16_tflops burst (%s)" % ("of measured" if peak_src == "measured" else "of fallback")}
+    roof["traffic"] = known_traffic(kern, prob.cfg["workload"])
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if prob.xfmt == "bf16" else "f32", "data": "synthetic",
+            "config": config_block(prob, args.config, {"path": path_used,
+                                                        "touched_experts": acc["touched"]}),
+            "roofline": roof,
+            "layer": {"algorithmic_bytes": acc["layer_bytes"], "algorithmic_flops": acc["layer_flops"],
+                      "hbm_frac_of_step": acc["layer_bytes"] / (step_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                      "kernels_ms": {n: round(t / max(c, 1), 5) for n, (c, t) in stages.items()}},
+            "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT,
+                    "h2d_bytes_per_step": int(x.numel() * x.element_size()),
+                    "d2h_bytes_per_step": int(y.numel() * y.element_size())},
+            "gpu_launches": int(launches),
+            "clocks": clocks.summary()}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample = time_oracle(prob, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    barrier()
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=2, choices=sorted(synth.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", default="auto", choices=["auto", "gemv", "gemm"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,176 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) routed mixture-of-experts layer.
+ *
+ * The layer, as the pages describe it:
+ *   router   logits = W_r x (fp32); sigmoid scores with a selection bias, the
+ *            top k chosen on score + bias, weights = the chosen SCORES
+ *            renormalised and multiplied by a scale (2.446 for Kimi-Linear) --
+ *            Kimi-Linear-48B-A3B LiteRT-LM details page, Conversion notes,
+ *            mixture-of-experts bullet; CMF code specialist page, step 1 ("the
+ *            sigmoid MoE router with its selection bias").  Or softmax, top k,
+ *            renormalise (Qwen3-30B-A3B LiteRT-LM card, Conversion Notes).
+ *   experts  only the k routed experts run for a token; each is a SiLU-gated
+ *            FFN  o = W_down (SiLU(W_gate x) * (W_up x))  (Qwen3 card,
+ *            Conversion Notes; the moe op's activation 'silu').
+ *   combine  y = sum over the k slots of weight * o, in slot order.  The
+ *            residual add stays outside the op (Qwen3 card, moe_fusion_guard
+ *            bullet).
+ *   storage  experts fp32, bf16, int8 with one fp32 scale per output row and
+ *            expert (Kimi details page, quantization bullet), or int4 in blocks
+ *            of 32 along the reduction axis with fp32 scales (Qwen3 card,
+ *            Available Artifacts table).
+ *   mask     an optional runtime expert mask: masked experts are never chosen;
+ *            this equals slicing the router rows, the bias and the experts
+ *            (CMF page, Defrag step).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, row-major,
+ *     and must be 16-byte aligned (the workspace 256-byte aligned).  Nothing
+ *     is allocated by moe_route / moe_forward: scratch comes from the caller's
+ *     workspace (size from moe_workspace_size).
+ *   - Work is enqueued asynchronously on `stream`; no entry point synchronises
+ *     except moe_device_flags and moe_stage_times (documented there).
+ *   - Arguments are validated on the host before anything is launched; a
+ *     non-OK status means nothing was enqueued, and moe_last_error() returns a
+ *     message for the calling thread.
+ *   - Problems found in DATA on the device (an expert index out of range in
+ *     caller-provided routing, fewer than k selectable experts, a non-finite
+ *     router logit) cannot be reported synchronously; kernels set bits in a
+ *     per-device sticky word read by moe_device_flags().  No kernel traps.
+ *   - The current CUDA device is the one the pointers live on.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size or enum value */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid but not built: e.g. an activation other than SiLU */
+  MOE_ERR_WORKSPACE = 3,    /* workspace missing or smaller than moe_workspace_size */
+  MOE_ERR_CUDA = 4          /* a CUDA launch or runtime call failed */
+} moe_status;
+
+typedef enum {
+  MOE_ROUTER_SIGMOID_BIAS = 0, /* key = sigmoid(l) + b, weight from sigmoid(l) */
+  MOE_ROUTER_SOFTMAX = 1       /* key = softmax(l) over active experts */
+} moe_router_kind;
+
+typedef enum {
+  MOE_W_F32 = 0,
+  MOE_W_BF16 = 1,
+  MOE_W_INT8_ROW = 2, /* int8, one fp32 scale per (expert, output row) */
+  MOE_W_INT4_B32 = 3  /* int4 two's complement, 2 per byte (low nibble = even
+                         column), one fp32 scale per 32 columns */
+} moe_wfmt;
+
+typedef enum { MOE_X_F32 = 0, MOE_X_BF16 = 1 } moe_xfmt;
+
+typedef enum {
+  MOE_ACT_SILU = 0,
+  MOE_ACT_GELU_TANH = 1 /* named by the pages' moe op; rejected with MOE_ERR_UNSUPPORTED */
+} moe_act;
+
+typedef enum {
+  MOE_PATH_AUTO = 0, /* pick by tokens per expert and formats */
+  MOE_PATH_GEMV = 1, /* weight-streaming split GEMV (any format) */
+  MOE_PATH_GEMM = 2  /* tcgen05 grouped GEMM (bf16 x; bf16/int8/int4 weights) */
+} moe_path;
+
+/*
+ * Layer description.  Shapes: x [T, H]; W_r [E, H] fp32; b [E] fp32 or NULL
+ * (zero bias); expert_mask [E] uint8 (1 = active) or NULL (all active).
+ *   W_gate, W_up : [E, I, H]   (int4: [E, I, H/2] bytes)
+ *   W_down       : [E, H, I]   (int4: [E, H, I/2] bytes)
+ *   s_gate, s_up : int8 [E, I];  int4 [E, I, H/32];  otherwise NULL
+ *   s_down       : int8 [E, H];  int4 [E, H, I/32];  otherwise NULL
+ * Limits: H, I multiples of 64; 1 <= k <= 32; k <= E <= 1024.
+ */
+typedef struct {
+  int32_t H, I, E, k;
+  int32_t router; /* moe_router_kind */
+  int32_t act;    /* moe_act */
+  int32_t wfmt;   /* moe_wfmt */
+  int32_t xfmt;   /* moe_xfmt (also the dtype of y) */
+  int32_t path;   /* moe_path */
+  float scale;    /* multiplies the renormalised weights: 2.446 Kimi, 1 Qwen3 */
+  const float* W_r;
+  const float* b;
+  const uint8_t* expert_mask;
+  const void* W_gate;
+  const void* W_up;
+  const void* W_down;
+  const float* s_gate;
+  const float* s_up;
+  const float* s_down;
+} moe_desc;
+
+/* Bytes of workspace moe_route and moe_forward need for T tokens (one buffer
+ * serves both; calls on one stream may reuse it). */
+MOE_API moe_status moe_workspace_size(const moe_desc* d, int32_t T, size_t* bytes);
+
+/*
+ * Router: topk_idx [T, k] int32 and topk_w [T, k] fp32, slots in descending
+ * key order with ties to the lower expert index.  Logits are fp32 sums; the
+ * softmax router selects on the logits, whose order equals the softmax's.
+ * Tokens with fewer than k selectable experts get idx -1 / w 0 in the
+ * unfilled slots and raise MOE_FLAG_TOO_FEW_ACTIVE.
+ */
+MOE_API moe_status moe_route(const moe_desc* d, const void* x, int32_t T, int32_t* topk_idx, float* topk_w,
+                     void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Experts + combine under a given routing (from moe_route or the caller):
+ * y [T, H] in x's dtype, y[t] = sum_j topk_w[t, j] * FFN_{topk_idx[t, j]}(x[t])
+ * summed in slot order in fp32, rounded once.  Slots whose index is outside
+ * [0, E) contribute nothing and raise MOE_FLAG_BAD_EXPERT_INDEX.
+ */
+MOE_API moe_status moe_forward(const moe_desc* d, const void* x, int32_t T, const int32_t* topk_idx,
+                       const float* topk_w, void* y, void* workspace, size_t ws_bytes,
+                       cudaStream_t stream);
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+MOE_API const char* moe_last_error(void);
+
+/* Device data-error flags (bits below) of the current device.  Synchronises
+ * the device.  clear != 0 resets the word after reading. */
+#define MOE_FLAG_BAD_EXPERT_INDEX 0x1u
+#define MOE_FLAG_TOO_FEW_ACTIVE 0x2u
+#define MOE_FLAG_NONFINITE_LOGIT 0x4u
+MOE_API moe_status moe_device_flags(uint32_t* flags, int32_t clear);
+
+/* Number of kernels this library has launched in this process. */
+MOE_API uint64_t moe_launch_count(void);
+
+/*
+ * Optional per-kernel timing: when enabled, every kernel launch is bracketed
+ * by CUDA events on its stream.  moe_stage_times() waits for those events and
+ * returns, per kernel name, the number of launches and the summed duration in
+ * ms since the previous call (then resets).  Off by default.
+ */
+typedef struct {
+  char name[32];
+  int32_t launches;
+  float total_ms;
+} moe_stage_time;
+MOE_API moe_status moe_stage_timing(int32_t enable);
+MOE_API moe_status moe_stage_times(moe_stage_time* out, int32_t capacity, int32_t* count);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -1,0 +1,59 @@
+// Host-side interface between the C ABI (moe_api.cu) and the kernel launchers.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// Tokens are routed in chunks of this many (token, slot) pairs when building
+// the expert-sorted order.
+constexpr int kPairChunk = 1024;
+
+// Split of the router's reduction over H into S partial sums (summed in a
+// fixed order by the top-k kernel).  Depends on T only, so a masked layer and
+// its sliced twin compute bit-identical logits.
+int router_splits(int T);
+
+// Device scratch carved from the caller's workspace.
+struct Workspace {
+  float* logits;      // [S, T, E] partial router logits
+  int32_t* chunk_hist;  // [NC, E] pairs per expert per chunk (then chunk bases)
+  int32_t* counts;    // [E]
+  int32_t* offsets;   // [E + 1] start of each expert in the sorted order
+  int32_t* touched;   // [E] experts with count > 0, ascending; touched[E] unused
+  int32_t* meta;      // [16] small device scalars (meta[0] = number of touched experts)
+  int32_t* sorted_pair;  // [P] pair id (t * k + slot) at each sorted position
+  void* hbuf;         // [P, I] activations between the two projections (bf16, or fp32 for fp32 weights)
+  float* yp;          // [P, H] per-pair expert outputs times routing weight, indexed by pair id
+  void* xs;           // [P, H] bf16 tokens gathered in sorted order (tensor-core path)
+  size_t total;
+};
+
+Workspace carve_workspace(const moe_desc& d, int32_t T, void* base);
+
+// launch bookkeeping (counting + optional event timing), defined in moe_api.cu
+cudaError_t launch_done(const char* name, cudaStream_t s, void* begin_event);
+void* launch_start(const char* name, cudaStream_t s);
+
+// ---- launchers (each enqueues exactly one kernel) ----
+cudaError_t launch_router_logits(const moe_desc& d, const void* x, int T, float* partial, int S,
+                                 cudaStream_t s);
+cudaError_t launch_router_topk(const moe_desc& d, const float* partial, int S, int T, int32_t* idx,
+                               float* w, uint32_t* flags, cudaStream_t s);
+cudaError_t launch_pair_histogram(const int32_t* idx, int P, int E, int32_t* chunk_hist,
+                                  uint32_t* flags, cudaStream_t s);
+cudaError_t launch_expert_scan(int NC, int E, int32_t* chunk_hist, int32_t* counts, int32_t* offsets,
+                               int32_t* touched, int32_t* meta, cudaStream_t s);
+cudaError_t launch_pair_scatter(const int32_t* idx, int P, int E, const int32_t* chunk_hist,
+                                int32_t* sorted_pair, cudaStream_t s);
+cudaError_t launch_gemv_gateup(const moe_desc& d, const void* x, int k, const Workspace& ws,
+                               int num_sms, cudaStream_t s);
+cudaError_t launch_gemv_down(const moe_desc& d, const float* topk_w, int k, const Workspace& ws,
+                             int num_sms, cudaStream_t s);
+cudaError_t launch_combine(const moe_desc& d, const int32_t* idx, int T, const float* yp, void* y,
+                           cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,359 @@
+// C ABI of the routed-MoE library: argument validation, workspace carving,
+// kernel dispatch, error reporting, launch accounting and optional per-kernel
+// event timing.  Every step of the layer runs in this library's kernels; there
+// is no host compute path.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "internal.h"
+#include "moe.h"
+
+namespace moe {
+
+// ------------------------------------------------------------------ errors
+
+static thread_local std::string g_err;
+
+static moe_status fail(moe_status code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+static moe_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(MOE_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// ------------------------------------------------------------------ per-device state
+
+static __device__ uint32_t g_device_flags;
+
+struct DeviceState {
+  bool ready = false;
+  int num_sms = 0;
+  uint32_t* flags = nullptr;  // device address of g_device_flags on this device
+};
+static std::mutex g_dev_mu;
+static DeviceState g_dev[64];
+
+static moe_status device_state(DeviceState** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceState& st = g_dev[dev];
+  if (!st.ready) {
+    e = cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    e = cudaGetSymbolAddress(reinterpret_cast<void**>(&st.flags), g_device_flags);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(device flags)");
+    st.ready = true;
+  }
+  *out = &st;
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------------ launch accounting
+
+static std::atomic<uint64_t> g_launches{0};
+static std::atomic<int> g_timing{0};
+
+struct Pending {
+  char name[32];
+  cudaEvent_t begin, end;
+};
+static std::mutex g_time_mu;
+static std::vector<Pending> g_pending;
+static std::vector<cudaEvent_t> g_event_pool;
+
+static cudaEvent_t pool_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t ev = g_event_pool.back();
+    g_event_pool.pop_back();
+    return ev;
+  }
+  cudaEvent_t ev = nullptr;
+  cudaEventCreate(&ev);
+  return ev;
+}
+
+void* launch_start(const char* name, cudaStream_t s) {
+  (void)name;
+  if (!g_timing.load(std::memory_order_relaxed)) return nullptr;
+  std::lock_guard<std::mutex> lk(g_time_mu);
+  cudaEvent_t ev = pool_event();
+  if (ev) cudaEventRecord(ev, s);
+  return ev;
+}
+
+cudaError_t launch_done(const char* name, cudaStream_t s, void* begin_event) {
+  cudaError_t err = cudaGetLastError();
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (begin_event) {
+    std::lock_guard<std::mutex> lk(g_time_mu);
+    Pending p;
+    snprintf(p.name, sizeof(p.name), "%s", name);
+    p.begin = static_cast<cudaEvent_t>(begin_event);
+    p.end = pool_event();
+    if (p.end) {
+      cudaEventRecord(p.end, s);
+      g_pending.push_back(p);
+    } else {
+      g_event_pool.push_back(p.begin);
+    }
+  }
+  return err;
+}
+
+#define MOE_LAUNCH(name, stream, call)                         \
+  do {                                                         \
+    void* _ev = launch_start(name, stream);                    \
+    cudaError_t _e1 = (call);                                  \
+    cudaError_t _e2 = launch_done(name, stream, _ev);          \
+    if (_e1 != cudaSuccess) return cuda_fail(_e1, name);       \
+    if (_e2 != cudaSuccess) return cuda_fail(_e2, name);       \
+  } while (0)
+
+// ------------------------------------------------------------------ validation
+
+static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+static moe_status validate_desc(const moe_desc* d) {
+  if (!d) return fail(MOE_ERR_INVALID_ARG, "desc is NULL");
+  if (d->H <= 0 || d->I <= 0 || d->E <= 0 || d->k <= 0)
+    return fail(MOE_ERR_INVALID_ARG, "H, I, E, k must be positive (got %d, %d, %d, %d)", d->H, d->I, d->E, d->k);
+  if (d->H % 64 || d->I % 64) return fail(MOE_ERR_INVALID_ARG, "H and I must be multiples of 64 (got %d, %d)", d->H, d->I);
+  if (d->H > 8192 || d->I > 8192) return fail(MOE_ERR_UNSUPPORTED, "H and I are limited to 8192 (got %d, %d)", d->H, d->I);
+  if (d->E > 1024) return fail(MOE_ERR_UNSUPPORTED, "E is limited to 1024 (got %d)", d->E);
+  if (d->k > 32 || d->k > d->E) return fail(MOE_ERR_INVALID_ARG, "k must be <= min(E, 32) (got k=%d, E=%d)", d->k, d->E);
+  if (d->router != MOE_ROUTER_SIGMOID_BIAS && d->router != MOE_ROUTER_SOFTMAX)
+    return fail(MOE_ERR_INVALID_ARG, "unknown router kind %d", d->router);
+  if (d->act != MOE_ACT_SILU) {
+    if (d->act == MOE_ACT_GELU_TANH)
+      return fail(MOE_ERR_UNSUPPORTED, "unsupported activation 'gelu_tanh': this library builds SiLU only");
+    return fail(MOE_ERR_INVALID_ARG, "unknown activation %d", d->act);
+  }
+  if (d->wfmt < MOE_W_F32 || d->wfmt > MOE_W_INT4_B32) return fail(MOE_ERR_INVALID_ARG, "unknown weight format %d", d->wfmt);
+  if (d->xfmt != MOE_X_F32 && d->xfmt != MOE_X_BF16) return fail(MOE_ERR_INVALID_ARG, "unknown activation dtype %d", d->xfmt);
+  if (d->path < MOE_PATH_AUTO || d->path > MOE_PATH_GEMM) return fail(MOE_ERR_INVALID_ARG, "unknown path %d", d->path);
+  if (!isfinite(d->scale)) return fail(MOE_ERR_INVALID_ARG, "scale must be finite");
+  if (!d->W_r || !aligned(d->W_r, 16)) return fail(MOE_ERR_INVALID_ARG, "W_r must be a non-NULL 16-byte aligned device pointer");
+  if (!d->W_gate || !d->W_up || !d->W_down)
+    return fail(MOE_ERR_INVALID_ARG, "W_gate, W_up and W_down must be non-NULL");
+  if (!aligned(d->W_gate, 16) || !aligned(d->W_up, 16) || !aligned(d->W_down, 16))
+    return fail(MOE_ERR_INVALID_ARG, "expert weights must be 16-byte aligned");
+  const bool scaled = d->wfmt == MOE_W_INT8_ROW || d->wfmt == MOE_W_INT4_B32;
+  if (scaled && (!d->s_gate || !d->s_up || !d->s_down))
+    return fail(MOE_ERR_INVALID_ARG, "int8/int4 weights need s_gate, s_up and s_down");
+  if (scaled && (!aligned(d->s_gate, 4) || !aligned(d->s_up, 4) || !aligned(d->s_down, 4)))
+    return fail(MOE_ERR_INVALID_ARG, "scales must be 4-byte aligned");
+  return MOE_OK;
+}
+
+static moe_status validate_T(int32_t T, int k) {
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T must be >= 0 (got %d)", T);
+  if ((int64_t)T * k > (int64_t)1 << 30) return fail(MOE_ERR_UNSUPPORTED, "T*k above 2^30 (got T=%d, k=%d)", T, k);
+  return MOE_OK;
+}
+
+// The tensor-core path needs bf16 activations, non-fp32 weights and 128-row tiles.
+static bool gemm_capable(const moe_desc& d) {
+  return false;  // tcgen05 grouped GEMM not wired yet
+}
+
+static int choose_path(const moe_desc& d, int32_t T) {
+  if (d.path == MOE_PATH_GEMV) return MOE_PATH_GEMV;
+  if (d.path == MOE_PATH_GEMM) return MOE_PATH_GEMM;
+  const long long pairs = (long long)T * d.k;
+  if (gemm_capable(d) && pairs >= 16LL * d.E) return MOE_PATH_GEMM;
+  return MOE_PATH_GEMV;
+}
+
+// ------------------------------------------------------------------ workspace
+
+static size_t up256(size_t v) { return (v + 255) / 256 * 256; }
+
+static void layout(const moe_desc& d, int32_t T, size_t off[10], size_t* total) {
+  const size_t P = (size_t)T * d.k, E = d.E;
+  const size_t S = router_splits(T);
+  const size_t NC = (P + kPairChunk - 1) / kPairChunk;
+  const size_t hbytes = d.wfmt == MOE_W_F32 ? 4 : 2;
+  const size_t xs_bytes = (d.xfmt == MOE_X_BF16 && d.wfmt != MOE_W_F32) ? P * d.H * 2 : 0;
+  const size_t sizes[10] = {S * T * E * 4, (NC ? NC : 1) * E * 4, E * 4, (E + 1) * 4, (E + 1) * 4, 16 * 4,
+                            P * 4, P * d.I * hbytes, P * d.H * 4, xs_bytes};
+  size_t o = 0;
+  for (int i = 0; i < 10; ++i) {
+    off[i] = o;
+    o += up256(sizes[i]);
+  }
+  *total = o;
+}
+
+Workspace carve_workspace(const moe_desc& d, int32_t T, void* base) {
+  size_t off[10], total;
+  layout(d, T, off, &total);
+  char* b = static_cast<char*>(base);
+  Workspace w;
+  w.logits = reinterpret_cast<float*>(b + off[0]);
+  w.chunk_hist = reinterpret_cast<int32_t*>(b + off[1]);
+  w.counts = reinterpret_cast<int32_t*>(b + off[2]);
+  w.offsets = reinterpret_cast<int32_t*>(b + off[3]);
+  w.touched = reinterpret_cast<int32_t*>(b + off[4]);
+  w.meta = reinterpret_cast<int32_t*>(b + off[5]);
+  w.sorted_pair = reinterpret_cast<int32_t*>(b + off[6]);
+  w.hbuf = b + off[7];
+  w.yp = reinterpret_cast<float*>(b + off[8]);
+  w.xs = b + off[9];
+  w.total = total;
+  return w;
+}
+
+static moe_status check_ws(const moe_desc& d, int32_t T, void* ws, size_t ws_bytes) {
+  size_t off[10], need;
+  layout(d, T, off, &need);
+  if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL (need %zu bytes)", need);
+  if (!aligned(ws, 256)) return fail(MOE_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (ws_bytes < need) return fail(MOE_ERR_WORKSPACE, "workspace too small: %zu bytes given, %zu needed", ws_bytes, need);
+  return MOE_OK;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+// ====================================================================== C ABI
+
+extern "C" moe_status moe_workspace_size(const moe_desc* d, int32_t T, size_t* bytes) {
+  g_err.clear();
+  moe_status st = validate_desc(d);
+  if (st != MOE_OK) return st;
+  if ((st = validate_T(T, d->k)) != MOE_OK) return st;
+  if (!bytes) return fail(MOE_ERR_INVALID_ARG, "bytes is NULL");
+  size_t off[10];
+  layout(*d, T, off, bytes);
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_route(const moe_desc* d, const void* x, int32_t T, int32_t* topk_idx, float* topk_w,
+                                void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  g_err.clear();
+  moe_status st = validate_desc(d);
+  if (st != MOE_OK) return st;
+  if ((st = validate_T(T, d->k)) != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!x || !aligned(x, 16)) return fail(MOE_ERR_INVALID_ARG, "x must be a non-NULL 16-byte aligned device pointer");
+  if (!topk_idx || !topk_w || !aligned(topk_idx, 4) || !aligned(topk_w, 4))
+    return fail(MOE_ERR_INVALID_ARG, "topk_idx and topk_w must be non-NULL, 4-byte aligned");
+  if ((st = check_ws(*d, T, workspace, ws_bytes)) != MOE_OK) return st;
+  DeviceState* dev = nullptr;
+  if ((st = device_state(&dev)) != MOE_OK) return st;
+  const Workspace ws = carve_workspace(*d, T, workspace);
+  const int S = router_splits(T);
+  MOE_LAUNCH("router_logits", stream, launch_router_logits(*d, x, T, ws.logits, S, stream));
+  MOE_LAUNCH("router_topk", stream, launch_router_topk(*d, ws.logits, S, T, topk_idx, topk_w, dev->flags, stream));
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_forward(const moe_desc* d, const void* x, int32_t T, const int32_t* topk_idx,
+                                  const float* topk_w, void* y, void* workspace, size_t ws_bytes,
+                                  cudaStream_t stream) {
+  g_err.clear();
+  moe_status st = validate_desc(d);
+  if (st != MOE_OK) return st;
+  if ((st = validate_T(T, d->k)) != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!x || !aligned(x, 16)) return fail(MOE_ERR_INVALID_ARG, "x must be a non-NULL 16-byte aligned device pointer");
+  if (!y || !aligned(y, 16)) return fail(MOE_ERR_INVALID_ARG, "y must be a non-NULL 16-byte aligned device pointer");
+  if (!topk_idx || !topk_w || !aligned(topk_idx, 4) || !aligned(topk_w, 4))
+    return fail(MOE_ERR_INVALID_ARG, "topk_idx and topk_w must be non-NULL, 4-byte aligned");
+  if ((st = check_ws(*d, T, workspace, ws_bytes)) != MOE_OK) return st;
+  const int path = choose_path(*d, T);
+  if (path == MOE_PATH_GEMM && !gemm_capable(*d))
+    return fail(MOE_ERR_UNSUPPORTED,
+                "tensor-core path needs bf16 activations, bf16/int8/int4 weights and H, I multiples of 128");
+  DeviceState* dev = nullptr;
+  if ((st = device_state(&dev)) != MOE_OK) return st;
+  const Workspace ws = carve_workspace(*d, T, workspace);
+  const int P = T * d->k;
+  const int NC = (P + kPairChunk - 1) / kPairChunk;
+  MOE_LAUNCH("pair_histogram", stream, launch_pair_histogram(topk_idx, P, d->E, ws.chunk_hist, dev->flags, stream));
+  MOE_LAUNCH("expert_scan", stream,
+             launch_expert_scan(NC, d->E, ws.chunk_hist, ws.counts, ws.offsets, ws.touched, ws.meta, stream));
+  MOE_LAUNCH("pair_scatter", stream, launch_pair_scatter(topk_idx, P, d->E, ws.chunk_hist, ws.sorted_pair, stream));
+  MOE_LAUNCH("gemv_gateup", stream, launch_gemv_gateup(*d, x, d->k, ws, dev->num_sms, stream));
+  MOE_LAUNCH("gemv_down", stream, launch_gemv_down(*d, topk_w, d->k, ws, dev->num_sms, stream));
+  MOE_LAUNCH("combine", stream, launch_combine(*d, topk_idx, T, ws.yp, y, stream));
+  return MOE_OK;
+}
+
+extern "C" const char* moe_last_error(void) { return g_err.c_str(); }
+
+extern "C" moe_status moe_device_flags(uint32_t* flags, int32_t clear) {
+  g_err.clear();
+  if (!flags) return fail(MOE_ERR_INVALID_ARG, "flags is NULL");
+  DeviceState* dev = nullptr;
+  moe_status st = device_state(&dev);
+  if (st != MOE_OK) return st;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  e = cudaMemcpy(flags, dev->flags, sizeof(uint32_t), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading device flags");
+  if (clear) {
+    e = cudaMemset(dev->flags, 0, sizeof(uint32_t));
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "clearing device flags");
+  }
+  return MOE_OK;
+}
+
+extern "C" uint64_t moe_launch_count(void) { return g_launches.load(); }
+
+extern "C" moe_status moe_stage_timing(int32_t enable) {
+  g_timing.store(enable ? 1 : 0);
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_stage_times(moe_stage_time* out, int32_t capacity, int32_t* count) {
+  g_err.clear();
+  if (!count || (capacity > 0 && !out)) return fail(MOE_ERR_INVALID_ARG, "out/count is NULL");
+  std::lock_guard<std::mutex> lk(g_time_mu);
+  std::vector<moe_stage_time> agg;
+  cudaError_t first = cudaSuccess;
+  for (const Pending& p : g_pending) {
+    float ms = 0.f;
+    cudaError_t e = cudaEventSynchronize(p.end);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, p.begin, p.end);
+    if (e != cudaSuccess && first == cudaSuccess) first = e;
+    size_t i = 0;
+    for (; i < agg.size(); ++i)
+      if (strncmp(agg[i].name, p.name, sizeof(p.name)) == 0) break;
+    if (i == agg.size()) {
+      moe_stage_time t;
+      memset(&t, 0, sizeof(t));
+      snprintf(t.name, sizeof(t.name), "%s", p.name);
+      agg.push_back(t);
+    }
+    agg[i].launches += 1;
+    agg[i].total_ms += ms;
+    g_event_pool.push_back(p.begin);
+    g_event_pool.push_back(p.end);
+  }
+  g_pending.clear();
+  *count = (int32_t)agg.size();
+  for (int32_t i = 0; i < capacity && i < (int32_t)agg.size(); ++i) out[i] = agg[i];
+  if (first != cudaSuccess) return cuda_fail(first, "stage timing events");
+  return MOE_OK;
+}

@@ -1,0 +1,150 @@
+// Expert-sorted order of the (token, slot) pairs: histogram, scan, stable
+// counting-sort scatter.  "only the 8 routed experts are computed for each
+// token" (Qwen3-30B-A3B LiteRT-LM card, Conversion Notes): grouping the pairs
+// by expert lets each expert's weights be streamed once for all its tokens.
+//
+// Pair p = t * k + slot.  The pairs are cut into chunks of kPairChunk; every
+// kernel walks a chunk in pair order, so the result is a deterministic, stable
+// sort by expert (ties in pair order) with no order-dependent atomics.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+__global__ void __launch_bounds__(256) pair_histogram_kernel(const int32_t* __restrict__ idx, int P, int E,
+                                                             int32_t* __restrict__ chunk_hist,
+                                                             uint32_t* flags) {
+  extern __shared__ int32_t hist[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int p0 = blockIdx.x * kPairChunk, p1 = min(P, p0 + kPairChunk);
+  bool bad = false;
+  for (int p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
+    const int e = idx[p];
+    if (e >= 0 && e < E)
+      atomicAdd(&hist[e], 1);
+    else
+      bad = true;
+  }
+  if (bad) raise_flag(flags, MOE_FLAG_BAD_EXPERT_INDEX);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_hist[(size_t)blockIdx.x * E + e] = hist[e];
+}
+
+// exclusive prefix sum over the block (blockDim.x <= 1024); returns the block total in *total
+__device__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
+  const int lane = lane_id(), w = warp_id(), nw = blockDim.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int n = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += n;
+  }
+  if (lane == 31) warp_sums[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int s = lane < nw ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int n = __shfl_up_sync(0xFFFFFFFFu, s, off);
+      if (lane >= off) s += n;
+    }
+    if (lane < nw) warp_sums[lane] = s;  // inclusive over warps
+  }
+  __syncthreads();
+  const int before = (w > 0 ? warp_sums[w - 1] : 0) + incl - v;
+  *total = warp_sums[nw - 1];
+  __syncthreads();
+  return before;
+}
+
+// one block, one thread per expert: per-chunk bases, counts, offsets, touched list
+__global__ void __launch_bounds__(1024) expert_scan_kernel(int NC, int E, int32_t* __restrict__ chunk_hist,
+                                                           int32_t* __restrict__ counts,
+                                                           int32_t* __restrict__ offsets,
+                                                           int32_t* __restrict__ touched,
+                                                           int32_t* __restrict__ meta) {
+  __shared__ int warp_sums[32];
+  const int e = threadIdx.x;
+  int running = 0;
+  if (e < E) {
+    for (int c = 0; c < NC; ++c) {
+      const int v = chunk_hist[(size_t)c * E + e];
+      chunk_hist[(size_t)c * E + e] = running;
+      running += v;
+    }
+    counts[e] = running;
+  }
+  int total;
+  const int off = block_exclusive_scan(e < E ? running : 0, warp_sums, &total);
+  if (e < E) {
+    offsets[e] = off;
+    for (int c = 0; c < NC; ++c) chunk_hist[(size_t)c * E + e] += off;
+  }
+  if (e == 0) offsets[E] = total;
+  int ntouched;
+  const int tpos = block_exclusive_scan((e < E && running > 0) ? 1 : 0, warp_sums, &ntouched);
+  if (e < E && running > 0) touched[tpos] = e;
+  if (e == 0) {
+    meta[0] = ntouched;
+    meta[1] = total;
+  }
+}
+
+// one warp per chunk: stable positions in pair order
+__global__ void __launch_bounds__(128) pair_scatter_kernel(const int32_t* __restrict__ idx, int P, int E,
+                                                           const int32_t* __restrict__ chunk_base,
+                                                           int32_t* __restrict__ sorted_pair) {
+  extern __shared__ int32_t running_all[];
+  const int w = warp_id(), lane = lane_id();
+  const int c = blockIdx.x * (blockDim.x >> 5) + w;
+  int32_t* running = running_all + w * E;
+  const int nchunks = (P + kPairChunk - 1) / kPairChunk;
+  if (c >= nchunks) return;
+  for (int e = lane; e < E; e += 32) running[e] = chunk_base[(size_t)c * E + e];
+  __syncwarp();
+  const int p0 = c * kPairChunk, p1 = min(P, p0 + kPairChunk);
+  const unsigned lt = (1u << lane) - 1u;
+  for (int pb = p0; pb < p1; pb += 32) {
+    const int p = pb + lane;
+    int e = (p < p1) ? idx[p] : -1;
+    if (e < 0 || e >= E) e = -1;
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+    int pos = 0;
+    if (e >= 0) {
+      pos = running[e] + __popc(peers & lt);
+      sorted_pair[pos] = p;
+    }
+    __syncwarp();
+    if (e >= 0 && lane == 31 - __clz(peers)) running[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pair_histogram(const int32_t* idx, int P, int E, int32_t* chunk_hist, uint32_t* flags,
+                                  cudaStream_t s) {
+  const int NC = (P + kPairChunk - 1) / kPairChunk;
+  pair_histogram_kernel<<<NC, 256, E * sizeof(int32_t), s>>>(idx, P, E, chunk_hist, flags);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_expert_scan(int NC, int E, int32_t* chunk_hist, int32_t* counts, int32_t* offsets,
+                               int32_t* touched, int32_t* meta, cudaStream_t s) {
+  const int threads = ((E + 31) / 32) * 32;
+  expert_scan_kernel<<<1, threads, 0, s>>>(NC, E, chunk_hist, counts, offsets, touched, meta);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pair_scatter(const int32_t* idx, int P, int E, const int32_t* chunk_base, int32_t* sorted_pair,
+                                cudaStream_t s) {
+  const int NC = (P + kPairChunk - 1) / kPairChunk;
+  const int warps = 4;
+  pair_scatter_kernel<<<(NC + warps - 1) / warps, warps * 32, warps * E * sizeof(int32_t), s>>>(
+      idx, P, E, chunk_base, sorted_pair);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,238 @@
+// Router of the routed-MoE layer: fp32 logits, sigmoid+selection-bias or
+// softmax keys, warp-shuffle top-k, renormalised weights times the scale.
+//
+// "the router in plain ops (sigmoid scores, the top 8 chosen on the scores
+// plus the correction bias, weights renormalized and scaled by 2.446)" --
+// Kimi-Linear LiteRT-LM details page, Conversion notes; "The router, its
+// softmax, the top 8 and their renormalization" -- Qwen3-30B-A3B LiteRT-LM
+// card, Conversion Notes.  Masked experts are never selectable (CMF page,
+// Defrag step: runtime expert mask).
+//
+// Two kernels:
+//   router_logits_kernel  tiled SIMT fp32 GEMM, partial[s][t][e] over S splits
+//                         of the H reduction (S chosen from T so small batches
+//                         still fill the GPU);
+//   router_topk_kernel    one warp per token: sums the S partials in a fixed
+//                         order, forms keys, selects k by repeated warp argmax
+//                         (key descending, expert index ascending), and
+//                         renormalises.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+int router_splits(int T) {
+  if (T <= 64) return 8;
+  if (T <= 256) return 4;
+  if (T <= 2048) return 2;
+  return 1;
+}
+
+namespace {
+
+constexpr int kBT = 64, kBE = 64, kBK = 32;
+
+template <bool XBF16>
+__global__ void __launch_bounds__(256) router_logits_kernel(const void* __restrict__ x,
+                                                            const float* __restrict__ Wr, int T, int H,
+                                                            int E, int kc, float* __restrict__ partial) {
+  __shared__ __align__(16) float xs[kBK][kBT + 4];
+  __shared__ __align__(16) float wsm[kBK][kBE + 4];
+  const int t0 = blockIdx.x * kBT, e0 = blockIdx.y * kBE, s = blockIdx.z;
+  const int kb = s * kc, ke = min(H, kb + kc);
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;  // output micro-tile: experts 4*tx.., tokens 4*ty..
+  const int lr = tid & 63, lq = (tid >> 6) * 8;  // loader: row lr, 8 columns from lq
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+  for (int k0 = kb; k0 < ke; k0 += kBK) {
+    float xv[8], wv[8];
+    const int t = t0 + lr;
+    if (t < T) {
+      if (XBF16) {
+        const uint4 v = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + (size_t)t * H + k0 + lq);
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          xv[2 * j] = bf16_to_f32(u[j] & 0xFFFFu);
+          xv[2 * j + 1] = bf16_to_f32(u[j] >> 16);
+        }
+      } else {
+        const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(x) + (size_t)t * H + k0 + lq);
+        const float4 a = p[0], b = p[1];
+        xv[0] = a.x; xv[1] = a.y; xv[2] = a.z; xv[3] = a.w;
+        xv[4] = b.x; xv[5] = b.y; xv[6] = b.z; xv[7] = b.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) xv[j] = 0.f;
+    }
+    const int e = e0 + lr;
+    if (e < E) {
+      const float4* p = reinterpret_cast<const float4*>(Wr + (size_t)e * H + k0 + lq);
+      const float4 a = p[0], b = p[1];
+      wv[0] = a.x; wv[1] = a.y; wv[2] = a.z; wv[3] = a.w;
+      wv[4] = b.x; wv[5] = b.y; wv[6] = b.z; wv[7] = b.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) wv[j] = 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      xs[lq + j][lr] = xv[j];
+      wsm[lq + j][lr] = wv[j];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kBK; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
+      const float4 b = *reinterpret_cast<const float4*>(&wsm[kk][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty * 4 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx * 4 + j;
+      if (e < E) partial[((size_t)s * T + t) * E + e] = acc[i][j];
+    }
+  }
+}
+
+// (key, expert) ordering: larger key first, then smaller expert index
+__device__ __forceinline__ bool better(float ka, int ea, float kb, int eb) {
+  return ka > kb || (ka == kb && ea < eb);
+}
+
+template <int PER_LANE>
+__global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ partial, int S, int T,
+                                                          int E, int k, int router,
+                                                          const float* __restrict__ bias,
+                                                          const uint8_t* __restrict__ mask, float scale,
+                                                          int32_t* __restrict__ idx, float* __restrict__ wout,
+                                                          uint32_t* flags) {
+  const int t = blockIdx.x * (blockDim.x >> 5) + warp_id();
+  if (t >= T) return;
+  const int lane = lane_id();
+  float logit[PER_LANE], key[PER_LANE];
+  uint32_t avail = 0;
+  bool bad = false;
+#pragma unroll
+  for (int j = 0; j < PER_LANE; ++j) {
+    const int e = lane + 32 * j;
+    logit[j] = 0.f;
+    key[j] = -INFINITY;
+    if (e < E) {
+      float l = 0.f;
+      for (int s = 0; s < S; ++s) l += partial[((size_t)s * T + t) * E + e];
+      logit[j] = l;
+      const bool active = (mask == nullptr) || (mask[e] != 0);
+      if (!isfinite(l)) {
+        bad = true;
+      } else if (active) {
+        key[j] = (router == MOE_ROUTER_SIGMOID_BIAS) ? sigmoidf_acc(l) + (bias ? bias[e] : 0.f) : l;
+        avail |= 1u << j;
+      }
+    }
+  }
+  if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) raise_flag(flags, MOE_FLAG_NONFINITE_LOGIT);
+
+  int my_e = -1;
+  float my_r = 0.f;
+  for (int slot = 0; slot < k; ++slot) {
+    float bk = -INFINITY;
+    int be = 0x7FFFFFFF;
+#pragma unroll
+    for (int j = 0; j < PER_LANE; ++j) {
+      if ((avail >> j) & 1u) {
+        const int e = lane + 32 * j;
+        if (better(key[j], e, bk, be)) {
+          bk = key[j];
+          be = e;
+        }
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ok = __shfl_xor_sync(0xFFFFFFFFu, bk, off);
+      const int oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
+      if (better(ok, oe, bk, be)) {
+        bk = ok;
+        be = oe;
+      }
+    }
+    const bool found = be != 0x7FFFFFFF;
+    float r = 0.f;
+    if (found && (be & 31) == lane) {
+      const int jj = be >> 5;
+#pragma unroll
+      for (int j = 0; j < PER_LANE; ++j)
+        if (j == jj) {
+          r = (router == MOE_ROUTER_SIGMOID_BIAS) ? sigmoidf_acc(logit[j]) : logit[j];
+          avail &= ~(1u << j);
+        }
+    }
+    r = __shfl_sync(0xFFFFFFFFu, r, found ? (be & 31) : 0);
+    if (lane == slot) {
+      my_e = found ? be : -1;
+      my_r = r;
+    }
+    if (!found && lane == 0) raise_flag(flags, MOE_FLAG_TOO_FEW_ACTIVE);
+  }
+  // renormalise over the chosen slots (softmax: exp relative to the best logit,
+  // which the full softmax denominator cancels against)
+  const float top = __shfl_sync(0xFFFFFFFFu, my_r, 0);
+  float v = 0.f;
+  if (lane < k && my_e >= 0) v = (router == MOE_ROUTER_SIGMOID_BIAS) ? my_r : expf(my_r - top);
+  float total = v;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) total += __shfl_xor_sync(0xFFFFFFFFu, total, off);
+  if (lane < k) {
+    idx[(size_t)t * k + lane] = my_e;
+    wout[(size_t)t * k + lane] = (my_e >= 0 && total > 0.f) ? v / total * scale : 0.f;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_router_logits(const moe_desc& d, const void* x, int T, float* partial, int S,
+                                 cudaStream_t s) {
+  int kc = (d.H + S - 1) / S;
+  kc = (kc + kBK - 1) / kBK * kBK;
+  dim3 grid((T + kBT - 1) / kBT, (d.E + kBE - 1) / kBE, S);
+  if (d.xfmt == MOE_X_BF16)
+    router_logits_kernel<true><<<grid, 256, 0, s>>>(x, d.W_r, T, d.H, d.E, kc, partial);
+  else
+    router_logits_kernel<false><<<grid, 256, 0, s>>>(x, d.W_r, T, d.H, d.E, kc, partial);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_topk(const moe_desc& d, const float* partial, int S, int T, int32_t* idx,
+                               float* w, uint32_t* flags, cudaStream_t s) {
+  const int warps = 8;
+  dim3 grid((T + warps - 1) / warps);
+  if (d.E <= 256)
+    router_topk_kernel<8><<<grid, warps * 32, 0, s>>>(partial, S, T, d.E, d.k, d.router, d.b, d.expert_mask,
+                                                      d.scale, idx, w, flags);
+  else
+    router_topk_kernel<32><<<grid, warps * 32, 0, s>>>(partial, S, T, d.E, d.k, d.router, d.b,
+                                                       d.expert_mask, d.scale, idx, w, flags);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,100 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/moe.h declares, and rejects bad arguments with the
+documented status before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mixture_experts_layer_31_b200 as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_entry_points():
+    names = []
+    for f in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if f.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", f)).read()
+            names += re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", txt)
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_entry_points()
+    assert set(moe.EXPORTS) <= set(names)
+    lib = ctypes.CDLL(moe.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def _desc(**kw):
+    d = moe.moe_desc()
+    d.H, d.I, d.E, d.k = 256, 128, 16, 4
+    d.router, d.act, d.wfmt, d.xfmt, d.path, d.scale = 0, 0, moe.MOE_W_BF16, moe.MOE_X_BF16, 0, 2.446
+    fake = 1 << 20  # never dereferenced: validation and sizing only
+    d.W_r = d.W_gate = d.W_up = d.W_down = fake
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+def test_workspace_size_grows_with_tokens():
+    a = moe.moe_workspace_size(_desc(), 16)
+    b = moe.moe_workspace_size(_desc(), 1024)
+    assert 0 < a < b and a % 256 == 0
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("H", 100, moe.MOE_ERR_INVALID_ARG),
+    ("I", 0, moe.MOE_ERR_INVALID_ARG),
+    ("k", 17, moe.MOE_ERR_INVALID_ARG),
+    ("k", 33, moe.MOE_ERR_INVALID_ARG),
+    ("E", 2048, moe.MOE_ERR_UNSUPPORTED),
+    ("act", moe.MOE_ACT_GELU_TANH, moe.MOE_ERR_UNSUPPORTED),
+    ("act", 7, moe.MOE_ERR_INVALID_ARG),
+    ("router", 5, moe.MOE_ERR_INVALID_ARG),
+    ("wfmt", 9, moe.MOE_ERR_INVALID_ARG),
+    ("W_r", None, moe.MOE_ERR_INVALID_ARG),
+    ("W_gate", (1 << 20) + 4, moe.MOE_ERR_INVALID_ARG),
+    ("wfmt", moe.MOE_W_INT8_ROW, moe.MOE_ERR_INVALID_ARG),  # int8 without scales
+])
+def test_invalid_descriptors_are_rejected(field, value, status):
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_workspace_size(_desc(**{field: value}), 16)
+    assert ei.value.status == status
+    assert moe.moe_last_error()
+
+
+def test_gelu_message_names_the_activation():
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_workspace_size(_desc(act=moe.MOE_ACT_GELU_TANH), 16)
+    assert "gelu_tanh" in str(ei.value)
+
+
+def test_route_and_forward_validate_before_launch():
+    d = _desc()
+    with pytest.raises(moe.MoeError) as ei:  # NULL x
+        moe.moe_route(d, None, 16, 1 << 20, 1 << 20, 1 << 20, 1 << 30)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+    with pytest.raises(moe.MoeError) as ei:  # workspace too small
+        moe.moe_route(d, 1 << 20, 16, 1 << 20, 1 << 20, 1 << 20, 256)
+    assert ei.value.status == moe.MOE_ERR_WORKSPACE
+    with pytest.raises(moe.MoeError) as ei:  # misaligned workspace
+        moe.moe_forward(d, 1 << 20, 16, 1 << 20, 1 << 20, 1 << 20, (1 << 20) + 64, 1 << 30)
+    assert ei.value.status == moe.MOE_ERR_WORKSPACE
+    with pytest.raises(moe.MoeError) as ei:  # negative T
+        moe.moe_forward(d, 1 << 20, -1, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 30)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+    # T = 0 is a valid no-op that launches nothing
+    n = moe.moe_launch_count()
+    moe.moe_route(d, 1 << 20, 0, 1 << 20, 1 << 20, None, 0)
+    moe.moe_forward(d, 1 << 20, 0, 1 << 20, 1 << 20, 1 << 20, None, 0)
+    assert moe.moe_launch_count() == n
+
+
+def test_header_declares_citations_and_ownership():
+    txt = open(os.path.join(ROOT, "include", "moe.h")).read()
+    for needle in ("Conversion notes", "Defrag", "owned by the caller", "MOE_ERR_UNSUPPORTED"):
+        assert needle in txt

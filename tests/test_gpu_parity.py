@@ -1,0 +1,175 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle on
+every workload, at sizes the oracle finishes in seconds (several tiles, ragged
+tails) and at the full workload sizes on sampled tokens."""
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_layer_31_b200 as moe
+import oracle
+import synth
+from gpu_util import judge, layer_from_problem, run, x_to_device
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+PATHS = {"auto": moe.MOE_PATH_AUTO, "gemv": moe.MOE_PATH_GEMV}
+
+# small variants of each workload: same formats/routers, shapes the oracle runs in seconds
+SMALL = {
+    "tiny-fp32": (1, {}),
+    "kimi-bf16-small": (2, dict(T=37, H=256, E=32, I=192)),
+    "kimi-int8-small": (3, dict(T=203, H=384, E=24, I=256)),
+    "qwen3-int4-small": (4, dict(T=150, H=256, E=16, I=128)),
+    "skew-masked-int8-small": (5, dict(T=301, H=256, E=40, I=128, n_active=23, bias=("skew", 0.15))),
+}
+
+
+@pytest.fixture(autouse=True)
+def _clear_flags():
+    moe.moe_device_flags(clear=True)
+    yield
+    assert moe.moe_device_flags(clear=True) == 0, "kernels raised a device data-error flag"
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_workloads(name, path):
+    cid, over = SMALL[name]
+    prob = synth.make_problem(cid, **over)
+    _, _, y, idx, w = run(prob, PATHS[path])
+    rep = judge(prob, y, idx, w)
+    assert rep["near_ties"] <= max(2, prob.T // 20)
+
+
+def test_tiny_fp32_full_tolerance():
+    prob = synth.make_problem(1)
+    _, _, y, idx, w = run(prob)
+    rep = judge(prob, y, idx, w, tol=1e-5)
+    assert rep["rel_l2"] <= 1e-5
+
+
+def test_kimi_decode_bf16_full():
+    """The decode workload at full size, every token."""
+    prob = synth.make_problem(2)
+    _, _, y, idx, w = run(prob)
+    judge(prob, y, idx, w)
+
+
+@pytest.mark.parametrize("cid,n_sample", [(3, 40), (4, 96), (5, 40)])
+def test_full_workloads_sampled(cid, n_sample):
+    """Full-size prefill workloads, the same launch as the benchmark; the oracle
+    checks a seeded sample of tokens (first, last and random ones)."""
+    prob = synth.make_problem(cid)
+    _, _, y, idx, w = run(prob)
+    rng = np.random.default_rng(cid)
+    toks = np.unique(np.concatenate([[0, prob.T - 1], rng.choice(prob.T, n_sample, replace=False)]))
+    judge(prob, y, idx, w, tokens=toks)
+    if prob.mask is not None:
+        assert prob.mask[idx.cpu().numpy()].all()
+
+
+def test_deterministic_repeat():
+    prob = synth.make_problem(3, T=257, H=256, E=16, I=128)
+    layer, x, y1, i1, w1 = run(prob)
+    y2, i2, w2 = layer(x)
+    torch.cuda.synchronize()
+    assert torch.equal(i1, i2) and torch.equal(w1, w2)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+def test_mask_equals_slice_bit_identical():
+    """Masking experts equals slicing router rows, bias and experts (CMF page,
+    Defrag step) -- bit for bit on the GPU as well."""
+    prob = synth.make_problem(5, T=180, H=256, E=48, I=128, n_active=29, bias=("skew", 0.2))
+    act = np.nonzero(prob.mask)[0]
+    sl = synth.Problem(cfg=prob.cfg, T=prob.T, H=prob.H, I=prob.I, E=len(act), k=prob.k, router=prob.router,
+                       scale=prob.scale, wfmt=prob.wfmt, xfmt=prob.xfmt, x=prob.x,
+                       W_r=np.ascontiguousarray(prob.W_r[act]), b=np.ascontiguousarray(prob.b[act]), mask=None,
+                       W_gate=np.ascontiguousarray(prob.W_gate[act]), W_up=np.ascontiguousarray(prob.W_up[act]),
+                       W_down=np.ascontiguousarray(prob.W_down[act]), s_gate=np.ascontiguousarray(prob.s_gate[act]),
+                       s_up=np.ascontiguousarray(prob.s_up[act]), s_down=np.ascontiguousarray(prob.s_down[act]))
+    _, _, y1, i1, w1 = run(prob)
+    _, _, y2, i2, w2 = run(sl)
+    assert np.array_equal(act[i2.cpu().numpy()], i1.cpu().numpy())
+    assert torch.equal(w1, w2)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+def test_single_token_and_k1():
+    prob = synth.make_problem(2, T=1, H=256, E=16, I=128)
+    _, _, y, idx, w = run(prob)
+    judge(prob, y, idx, w)
+    prob = synth.make_problem(3, T=33, H=256, E=16, I=128, k=1)
+    _, _, y, idx, w = run(prob)
+    judge(prob, y, idx, w)
+    assert np.allclose(w.cpu().numpy(), prob.scale)
+
+
+def test_all_experts_selected():
+    prob = synth.make_problem(4, T=20, H=256, E=8, I=128, k=8)
+    _, _, y, idx, w = run(prob)
+    judge(prob, y, idx, w)
+
+
+def test_caller_routing_all_to_one_expert():
+    """Every pair on one expert (maximal imbalance), under caller-provided routing."""
+    prob = synth.make_problem(3, T=300, H=256, E=16, I=128, k=2)
+    layer = layer_from_problem(prob)
+    x = x_to_device(prob)
+    idx = torch.full((prob.T, prob.k), 5, dtype=torch.int32, device="cuda")
+    idx[:, 1] = 11
+    w = torch.rand((prob.T, prob.k), device="cuda")
+    y = layer.forward(x, idx, w)
+    torch.cuda.synchronize()
+    ref = oracle.Oracle(prob).combine(range(prob.T), idx.cpu().numpy(), w.cpu().double().numpy())
+    rel = np.linalg.norm(y.double().cpu().numpy() - ref) / np.linalg.norm(ref)
+    assert rel < 5e-3
+
+
+def test_bad_expert_index_is_flagged_and_skipped():
+    prob = synth.make_problem(2, T=8, H=256, E=16, I=128, k=2)
+    layer = layer_from_problem(prob)
+    x = x_to_device(prob)
+    idx = torch.tensor([[1, 99]] * prob.T, dtype=torch.int32, device="cuda")
+    w = torch.ones((prob.T, prob.k), device="cuda")
+    y = layer.forward(x, idx, w)
+    assert moe.moe_device_flags(clear=True) & moe.MOE_FLAG_BAD_EXPERT_INDEX
+    ref = oracle.Oracle(prob).combine(range(prob.T), np.ones((prob.T, 1), np.int32) * 1, np.ones((prob.T, 1)))
+    rel = np.linalg.norm(y.double().cpu().numpy() - ref) / np.linalg.norm(ref)
+    assert rel < 5e-3
+
+
+def test_too_few_active_experts_is_flagged():
+    prob = synth.make_problem(5, T=4, H=256, E=16, I=128, n_active=5, k=8, bias=None)
+    layer = layer_from_problem(prob)
+    idx, w = layer.route(x_to_device(prob))
+    assert moe.moe_device_flags(clear=True) & moe.MOE_FLAG_TOO_FEW_ACTIVE
+    i = idx.cpu().numpy()
+    assert (i[:, :5] >= 0).all() and (i[:, 5:] == -1).all()
+    assert prob.mask[i[:, :5]].all()
+    np.testing.assert_allclose(w.cpu().numpy()[:, :5].sum(1), prob.scale, rtol=1e-5)
+
+
+def test_zero_tokens_is_a_noop():
+    prob = synth.make_problem(1)
+    layer = layer_from_problem(prob)
+    n = moe.moe_launch_count()
+    x = torch.empty((0, prob.H), device="cuda")
+    idx, w = layer.route(x)
+    layer.forward(x, idx, w)
+    assert moe.moe_launch_count() == n
+
+
+def test_stage_timing_reports_every_kernel():
+    prob = synth.make_problem(2, T=16, H=256, E=16, I=128)
+    layer = layer_from_problem(prob)
+    x = x_to_device(prob)
+    moe.moe_stage_timing(True)
+    try:
+        layer(x)
+        times = moe.moe_stage_times()
+    finally:
+        moe.moe_stage_timing(False)
+    for name in ("router_logits", "router_topk", "pair_histogram", "expert_scan", "pair_scatter", "combine"):
+        assert name in times and times[name][0] == 1 and times[name][1] > 0
