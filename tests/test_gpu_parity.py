@@ -135,7 +135,11 @@ def test_bad_expert_index_is_flagged_and_skipped():
     w = torch.ones((prob.T, prob.k), device="cuda")
     y = layer.forward(x, idx, w)
     assert moe.moe_device_flags(clear=True) & moe.MOE_FLAG_BAD_EXPERT_INDEX
-    ref = oracle.Oracle(prob).combine(range(prob.T), np.ones((prob.T, 1), np.int32) * 1, np.ones((prob.T, 1)))
+    # the invalid slot contributes nothing: same as expert 1 with weight 1 plus a zero-weight slot
+    ref_idx = np.ones((prob.T, prob.k), np.int32)
+    ref_w = np.zeros((prob.T, prob.k))
+    ref_w[:, 0] = 1.0
+    ref = oracle.Oracle(prob).combine(range(prob.T), ref_idx, ref_w)
     rel = np.linalg.norm(y.double().cpu().numpy() - ref) / np.linalg.norm(ref)
     assert rel < 5e-3
 
