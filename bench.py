@@ -257,7 +257,7 @@ def run_reference(args):
     rank, world = dist_init("gloo")
     if rank != 0:
         return 0
-    prob = synth.make_problem(args.config)
+    prob = synth.make_problem(args.config, **args.overrides)
     import oracle
     cores = cpu_threads()
     orc = oracle.Oracle(prob, nthreads=cores)
@@ -296,7 +296,7 @@ def run_ours(args):
     dist_init("nccl")
     import mixture_experts_layer_31_b200 as moe
     dev = torch.device("cuda", local)
-    prob = synth.make_problem(args.config)
+    prob = synth.make_problem(args.config, **args.overrides)
     path = {"auto": moe.MOE_PATH_AUTO, "gemv": moe.MOE_PATH_GEMV, "gemm": moe.MOE_PATH_GEMM}[args.path]
     layer = moe.MoELayer(H=prob.H, I=prob.I, E=prob.E, k=prob.k, router=prob.router, scale=prob.scale,
                          wfmt=prob.wfmt, xfmt=prob.xfmt, W_r=prob.W_r, b=prob.b, expert_mask=prob.mask,
@@ -394,8 +394,8 @@ def run_ours(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if prob.xfmt == "bf16" else "f32", "data": "synthetic",
-            "config": config_block(prob, args.config, {"path": path_used,
-                                                        "touched_experts": acc["touched"]}),
+            "config": config_block(prob, args.config, {"path": path_used, "touched_experts": acc["touched"],
+                                                        "overrides": args.overrides or None}),
             "roofline": roof,
             "layer": {"algorithmic_bytes": acc["layer_bytes"], "algorithmic_flops": acc["layer_flops"],
                       "hbm_frac_of_step": acc["layer_bytes"] / (step_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
@@ -427,7 +427,13 @@ def main(argv=None):
     ap.add_argument("--path", default="auto", choices=["auto", "gemv", "gemm"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--set", action="append", default=[], metavar="KEY=VAL",
+                    help="override a workload field (e.g. E=64) -- for small profiling cases; not a bench line")
     args = ap.parse_args(argv)
+    args.overrides = {}
+    for kv in args.set:
+        k_, v_ = kv.split("=", 1)
+        args.overrides[k_] = int(v_) if v_.lstrip("-").isdigit() else v_
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -6,8 +6,9 @@ carry the ABI's names and only marshal arguments; every step of the layer runs
 in the library's CUDA kernels.  ``MoELayer`` is a convenience wrapper that keeps
 device tensors (PyTorch is used for device memory and streams only).
 
-There is no CPU fallback: importing this package on a machine without the
-built library raises, and calls on a machine without a CUDA device fail.
+There is no CPU fallback: the first call into the library raises ImportError
+when ``libmoe_b200.so`` is not built, and calls on a machine without a CUDA
+device fail with MOE_ERR_CUDA.
 """
 from __future__ import annotations
 
@@ -81,48 +82,56 @@ def _load() -> ctypes.CDLL:
     return lib
 
 
-_lib = _load()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (loaded on first use; raises if it is not built)."""
+    global _lib
+    if _lib is None:
+        _lib = _load()
+    return _lib
 
 
 def _check(status: int):
     if status != MOE_OK:
-        raise MoeError(status, _lib.moe_last_error().decode())
+        raise MoeError(status, lib().moe_last_error().decode())
 
 
 # ---------------------------------------------------------------- ABI functions
 
 def moe_workspace_size(desc: moe_desc, T: int) -> int:
     n = ctypes.c_size_t(0)
-    _check(_lib.moe_workspace_size(ctypes.byref(desc), int(T), ctypes.byref(n)))
+    _check(lib().moe_workspace_size(ctypes.byref(desc), int(T), ctypes.byref(n)))
     return n.value
 
 
 def moe_route(desc: moe_desc, x: int, T: int, topk_idx: int, topk_w: int, workspace: int, ws_bytes: int,
               stream: int = 0) -> None:
-    _check(_lib.moe_route(ctypes.byref(desc), x, int(T), topk_idx, topk_w, workspace, int(ws_bytes), stream))
+    _check(lib().moe_route(ctypes.byref(desc), x, int(T), topk_idx, topk_w, workspace, int(ws_bytes), stream))
 
 
 def moe_forward(desc: moe_desc, x: int, T: int, topk_idx: int, topk_w: int, y: int, workspace: int,
                 ws_bytes: int, stream: int = 0) -> None:
-    _check(_lib.moe_forward(ctypes.byref(desc), x, int(T), topk_idx, topk_w, y, workspace, int(ws_bytes), stream))
+    _check(lib().moe_forward(ctypes.byref(desc), x, int(T), topk_idx, topk_w, y, workspace, int(ws_bytes), stream))
 
 
 def moe_last_error() -> str:
-    return _lib.moe_last_error().decode()
+    return lib().moe_last_error().decode()
 
 
 def moe_device_flags(clear: bool = False) -> int:
     v = ctypes.c_uint32(0)
-    _check(_lib.moe_device_flags(ctypes.byref(v), 1 if clear else 0))
+    _check(lib().moe_device_flags(ctypes.byref(v), 1 if clear else 0))
     return v.value
 
 
 def moe_launch_count() -> int:
-    return int(_lib.moe_launch_count())
+    return int(lib().moe_launch_count())
 
 
 def moe_stage_timing(enable: bool) -> None:
-    _check(_lib.moe_stage_timing(1 if enable else 0))
+    _check(lib().moe_stage_timing(1 if enable else 0))
 
 
 def moe_stage_times() -> dict:
@@ -130,7 +139,7 @@ def moe_stage_times() -> dict:
     cap = 64
     buf = (moe_stage_time * cap)()
     n = ctypes.c_int32(0)
-    _check(_lib.moe_stage_times(buf, cap, ctypes.byref(n)))
+    _check(lib().moe_stage_times(buf, cap, ctypes.byref(n)))
     return {buf[i].name.decode(): (int(buf[i].launches), float(buf[i].total_ms)) for i in range(min(n.value, cap))}
 
 
@@ -143,6 +152,7 @@ class MoELayer:
     def __init__(self, *, H, I, E, k, router, scale, wfmt, xfmt, W_r, W_gate, W_up, W_down, b=None,
                  expert_mask=None, s_gate=None, s_up=None, s_down=None, path=MOE_PATH_AUTO, device="cuda"):
         import torch
+        lib()  # fail loudly now if the CUDA library is missing
         self.torch = torch
         self.device = torch.device(device)
 
