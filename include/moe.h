@@ -143,6 +143,34 @@ MOE_API moe_status moe_forward(const moe_desc* d, const void* x, int32_t T, cons
                        const float* topk_w, void* y, void* workspace, size_t ws_bytes,
                        cudaStream_t stream);
 
+/*
+ * moe_forward without a workspace argument, for callers that cannot allocate
+ * device memory: a plugin host that owns every device buffer and hands the
+ * library no allocator, or a latency-bound loop that must not call cudaMalloc
+ * (which can synchronise the device) once it runs.  The pages describe no
+ * such entry point; it has no counterpart there.
+ *
+ * Scratch comes from one static device array of MOE_NOALLOC_SCRATCH_BYTES
+ * that this library holds on every GPU that loads it, until the process
+ * exits.  Inputs and outputs are still the caller's, exactly as for
+ * moe_forward, and the result is the same as moe_forward's.  Problems whose
+ * scratch (moe_workspace_size) exceeds the array -- roughly decode-sized
+ * batches fit -- are rejected with MOE_ERR_WORKSPACE and a message; nothing is
+ * launched then.  No cudaMalloc/cudaFree or other allocating call is made
+ * (leave moe_stage_timing off: the timing itself creates CUDA events).
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Every call shares the one array and it keeps
+ * the previous call's contents (nothing in it needs to start at zero: each
+ * call writes what it reads), so calls whose work overlaps on the GPU --
+ * several streams, or several host threads -- race on it and give wrong
+ * results; order them on one stream.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES (16u << 20)
+MOE_API moe_status moe_forward_noalloc(const moe_desc* d, const void* x, int32_t T, const int32_t* topk_idx,
+                                       const float* topk_w, void* y, cudaStream_t stream);
+
 /* Message for the last non-OK status returned on this thread ("" if none). */
 MOE_API const char* moe_last_error(void);
 

@@ -34,8 +34,9 @@ WFMT = {"f32": MOE_W_F32, "bf16": MOE_W_BF16, "int8": MOE_W_INT8_ROW, "int4": MO
 XFMT = {"f32": MOE_X_F32, "bf16": MOE_X_BF16}
 ROUTER = {"sigmoid": MOE_ROUTER_SIGMOID_BIAS, "softmax": MOE_ROUTER_SOFTMAX}
 
-EXPORTS = ("moe_workspace_size", "moe_route", "moe_forward", "moe_last_error", "moe_device_flags",
-           "moe_launch_count", "moe_stage_timing", "moe_stage_times")
+EXPORTS = ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_noalloc", "moe_last_error",
+           "moe_device_flags", "moe_launch_count", "moe_stage_timing", "moe_stage_times")
+MOE_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class MoeError(RuntimeError):
@@ -69,6 +70,7 @@ def _load() -> ctypes.CDLL:
     lib.moe_workspace_size.argtypes = [D, i32, ctypes.POINTER(sz)]
     lib.moe_route.argtypes = [D, vp, i32, vp, vp, vp, sz, vp]
     lib.moe_forward.argtypes = [D, vp, i32, vp, vp, vp, vp, sz, vp]
+    lib.moe_forward_noalloc.argtypes = [D, vp, i32, vp, vp, vp, vp]
     lib.moe_last_error.argtypes = []
     lib.moe_last_error.restype = ctypes.c_char_p
     lib.moe_device_flags.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
@@ -76,8 +78,8 @@ def _load() -> ctypes.CDLL:
     lib.moe_launch_count.restype = ctypes.c_uint64
     lib.moe_stage_timing.argtypes = [i32]
     lib.moe_stage_times.argtypes = [ctypes.POINTER(moe_stage_time), i32, ctypes.POINTER(i32)]
-    for f in ("moe_workspace_size", "moe_route", "moe_forward", "moe_device_flags", "moe_stage_timing",
-              "moe_stage_times"):
+    for f in ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_noalloc", "moe_device_flags",
+              "moe_stage_timing", "moe_stage_times"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -114,6 +116,13 @@ def moe_route(desc: moe_desc, x: int, T: int, topk_idx: int, topk_w: int, worksp
 def moe_forward(desc: moe_desc, x: int, T: int, topk_idx: int, topk_w: int, y: int, workspace: int,
                 ws_bytes: int, stream: int = 0) -> None:
     _check(lib().moe_forward(ctypes.byref(desc), x, int(T), topk_idx, topk_w, y, workspace, int(ws_bytes), stream))
+
+
+def moe_forward_noalloc(desc: moe_desc, x: int, T: int, topk_idx: int, topk_w: int, y: int,
+                        stream: int = 0) -> None:
+    """moe_forward with the library's static scratch instead of a workspace, for
+    callers that cannot allocate device memory (see include/moe.h)."""
+    _check(lib().moe_forward_noalloc(ctypes.byref(desc), x, int(T), topk_idx, topk_w, y, stream))
 
 
 def moe_last_error() -> str:

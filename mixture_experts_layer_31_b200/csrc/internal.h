@@ -34,6 +34,9 @@ struct Workspace {
 
 Workspace carve_workspace(const moe_desc& d, int32_t T, void* base);
 
+// set the calling thread's moe_last_error() message and return `code`
+moe_status report_error(moe_status code, const char* message);
+
 // launch bookkeeping (counting + optional event timing), defined in moe_api.cu
 cudaError_t launch_done(const char* name, cudaStream_t s, void* begin_event);
 void* launch_start(const char* name, cudaStream_t s);

@@ -32,6 +32,8 @@ static moe_status fail(moe_status code, const char* fmt, ...) {
   return code;
 }
 
+moe_status report_error(moe_status code, const char* message) { return fail(code, "%s", message); }
+
 static moe_status cuda_fail(cudaError_t e, const char* what) {
   return fail(MOE_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
