@@ -36,7 +36,8 @@
  *   - Problems found in DATA on the device (an expert index out of range in
  *     caller-provided routing, fewer than k selectable experts, a non-finite
  *     router logit) cannot be reported synchronously; kernels set bits in a
- *     per-device sticky word read by moe_device_flags().  No kernel traps.
+ *     per-device sticky word read by moe_device_flags().  No kernel traps, and
+ *     every wait inside a kernel is bounded in time (MOE_FLAG_TIMEOUT).
  *   - The current CUDA device is the one the pointers live on.
  */
 #ifndef MOE_B200_H
@@ -179,6 +180,7 @@ MOE_API const char* moe_last_error(void);
 #define MOE_FLAG_BAD_EXPERT_INDEX 0x1u
 #define MOE_FLAG_TOO_FEW_ACTIVE 0x2u
 #define MOE_FLAG_NONFINITE_LOGIT 0x4u
+#define MOE_FLAG_TIMEOUT 0x8u /* a kernel's bounded wait expired; its outputs are incomplete */
 MOE_API moe_status moe_device_flags(uint32_t* flags, int32_t clear);
 
 /* Number of kernels this library has launched in this process. */

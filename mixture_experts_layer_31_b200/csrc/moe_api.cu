@@ -172,32 +172,34 @@ static moe_status validate_T(int32_t T, int k) {
 }
 
 // The tensor-core path needs bf16 activations, non-fp32 weights and 128-row tiles.
-static bool gemm_capable(const moe_desc& d) {
-  return false;  // tcgen05 grouped GEMM not wired yet
-}
+static bool gemm_capable(const moe_desc& d) { return gemm_tc_supported(d); }
 
+// The tensor-core path streams weights with TMA and serves decode as well as
+// prefill; the SIMT GEMV path remains for fp32 layers and shapes the tensor
+// cores cannot tile.
 static int choose_path(const moe_desc& d, int32_t T) {
+  (void)T;
   if (d.path == MOE_PATH_GEMV) return MOE_PATH_GEMV;
   if (d.path == MOE_PATH_GEMM) return MOE_PATH_GEMM;
-  const long long pairs = (long long)T * d.k;
-  if (gemm_capable(d) && pairs >= 16LL * d.E) return MOE_PATH_GEMM;
-  return MOE_PATH_GEMV;
+  return gemm_capable(d) ? MOE_PATH_GEMM : MOE_PATH_GEMV;
 }
 
 // ------------------------------------------------------------------ workspace
 
 static size_t up256(size_t v) { return (v + 255) / 256 * 256; }
 
-static void layout(const moe_desc& d, int32_t T, size_t off[10], size_t* total) {
+constexpr int kRegions = 12;
+
+static void layout(const moe_desc& d, int32_t T, size_t off[kRegions], size_t* total) {
   const size_t P = (size_t)T * d.k, E = d.E;
   const size_t S = router_splits(T);
   const size_t NC = (P + kPairChunk - 1) / kPairChunk;
   const size_t hbytes = d.wfmt == MOE_W_F32 ? 4 : 2;
   const size_t xs_bytes = (d.xfmt == MOE_X_BF16 && d.wfmt != MOE_W_F32) ? P * d.H * 2 : 0;
-  const size_t sizes[10] = {S * T * E * 4, (NC ? NC : 1) * E * 4, E * 4, (E + 1) * 4, (E + 1) * 4, 16 * 4,
-                            P * 4, P * d.I * hbytes, P * d.H * 4, xs_bytes};
+  const size_t sizes[kRegions] = {S * T * E * 4, (NC ? NC : 1) * E * 4, E * 4, (E + 1) * 4, (E + 1) * 4, 16 * 4,
+                                  P * 4, P * d.I * hbytes, P * d.H * 4, xs_bytes, (E + 1) * 4, (E + 1) * 4};
   size_t o = 0;
-  for (int i = 0; i < 10; ++i) {
+  for (int i = 0; i < kRegions; ++i) {
     off[i] = o;
     o += up256(sizes[i]);
   }
@@ -205,7 +207,7 @@ static void layout(const moe_desc& d, int32_t T, size_t off[10], size_t* total) 
 }
 
 Workspace carve_workspace(const moe_desc& d, int32_t T, void* base) {
-  size_t off[10], total;
+  size_t off[kRegions], total;
   layout(d, T, off, &total);
   char* b = static_cast<char*>(base);
   Workspace w;
@@ -219,12 +221,14 @@ Workspace carve_workspace(const moe_desc& d, int32_t T, void* base) {
   w.hbuf = b + off[7];
   w.yp = reinterpret_cast<float*>(b + off[8]);
   w.xs = b + off[9];
+  w.group_base = reinterpret_cast<int32_t*>(b + off[10]);
+  w.tile_base = reinterpret_cast<int32_t*>(b + off[11]);
   w.total = total;
   return w;
 }
 
 static moe_status check_ws(const moe_desc& d, int32_t T, void* ws, size_t ws_bytes) {
-  size_t off[10], need;
+  size_t off[kRegions], need;
   layout(d, T, off, &need);
   if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL (need %zu bytes)", need);
   if (!aligned(ws, 256)) return fail(MOE_ERR_WORKSPACE, "workspace must be 256-byte aligned");
@@ -244,7 +248,7 @@ extern "C" moe_status moe_workspace_size(const moe_desc* d, int32_t T, size_t* b
   if (st != MOE_OK) return st;
   if ((st = validate_T(T, d->k)) != MOE_OK) return st;
   if (!bytes) return fail(MOE_ERR_INVALID_ARG, "bytes is NULL");
-  size_t off[10];
+  size_t off[kRegions];
   layout(*d, T, off, bytes);
   return MOE_OK;
 }
@@ -293,10 +297,17 @@ extern "C" moe_status moe_forward(const moe_desc* d, const void* x, int32_t T, c
   const int NC = (P + kPairChunk - 1) / kPairChunk;
   MOE_LAUNCH("pair_histogram", stream, launch_pair_histogram(topk_idx, P, d->E, ws.chunk_hist, dev->flags, stream));
   MOE_LAUNCH("expert_scan", stream,
-             launch_expert_scan(NC, d->E, ws.chunk_hist, ws.counts, ws.offsets, ws.touched, ws.meta, stream));
+             launch_expert_scan(NC, d->E, ws.chunk_hist, ws.counts, ws.offsets, ws.touched, ws.group_base,
+                                ws.tile_base, ws.meta, stream));
   MOE_LAUNCH("pair_scatter", stream, launch_pair_scatter(topk_idx, P, d->E, ws.chunk_hist, ws.sorted_pair, stream));
-  MOE_LAUNCH("gemv_gateup", stream, launch_gemv_gateup(*d, x, d->k, ws, dev->num_sms, stream));
-  MOE_LAUNCH("gemv_down", stream, launch_gemv_down(*d, topk_w, d->k, ws, dev->num_sms, stream));
+  if (path == MOE_PATH_GEMM) {
+    MOE_LAUNCH("gather_rows", stream, launch_gather_rows(*d, x, ws, P, dev->num_sms, stream));
+    MOE_LAUNCH("gemm_gateup", stream, launch_gemm_gateup(*d, ws, P, dev->num_sms, dev->flags, stream));
+    MOE_LAUNCH("gemm_down", stream, launch_gemm_down(*d, topk_w, ws, P, dev->num_sms, dev->flags, stream));
+  } else {
+    MOE_LAUNCH("gemv_gateup", stream, launch_gemv_gateup(*d, x, d->k, ws, dev->num_sms, dev->flags, stream));
+    MOE_LAUNCH("gemv_down", stream, launch_gemv_down(*d, topk_w, d->k, ws, dev->num_sms, dev->flags, stream));
+  }
   MOE_LAUNCH("combine", stream, launch_combine(*d, topk_idx, T, ws.yp, y, stream));
   return MOE_OK;
 }

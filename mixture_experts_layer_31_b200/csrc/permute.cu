@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(1024) expert_scan_kernel(int NC, int E, int32_
                                                            int32_t* __restrict__ counts,
                                                            int32_t* __restrict__ offsets,
                                                            int32_t* __restrict__ touched,
+                                                           int32_t* __restrict__ group_base,
+                                                           int32_t* __restrict__ tile_base,
                                                            int32_t* __restrict__ meta) {
   __shared__ int warp_sums[32];
   const int e = threadIdx.x;
@@ -86,9 +88,23 @@ __global__ void __launch_bounds__(1024) expert_scan_kernel(int NC, int E, int32_
   int ntouched;
   const int tpos = block_exclusive_scan((e < E && running > 0) ? 1 : 0, warp_sums, &ntouched);
   if (e < E && running > 0) touched[tpos] = e;
+  // token groups per touched expert, prefixed in touched (= ascending expert) order
+  const int groups = (e < E) ? (running + kGemvGroup - 1) / kGemvGroup : 0;
+  int ngroups;
+  const int gpos = block_exclusive_scan(groups, warp_sums, &ngroups);
+  if (e < E && running > 0) group_base[tpos] = gpos;
+  // token chunks of the tensor-core path, same order
+  const int chunks = (e < E) ? (running + kTileN - 1) / kTileN : 0;
+  int nchunks;
+  const int cpos = block_exclusive_scan(chunks, warp_sums, &nchunks);
+  if (e < E && running > 0) tile_base[tpos] = cpos;
   if (e == 0) {
     meta[0] = ntouched;
     meta[1] = total;
+    meta[2] = ngroups;
+    meta[3] = nchunks;
+    group_base[ntouched] = ngroups;
+    tile_base[ntouched] = nchunks;
   }
 }
 
@@ -132,9 +148,11 @@ cudaError_t launch_pair_histogram(const int32_t* idx, int P, int E, int32_t* chu
 }
 
 cudaError_t launch_expert_scan(int NC, int E, int32_t* chunk_hist, int32_t* counts, int32_t* offsets,
-                               int32_t* touched, int32_t* meta, cudaStream_t s) {
+                               int32_t* touched, int32_t* group_base, int32_t* tile_base, int32_t* meta,
+                               cudaStream_t s) {
   const int threads = ((E + 31) / 32) * 32;
-  expert_scan_kernel<<<1, threads, 0, s>>>(NC, E, chunk_hist, counts, offsets, touched, meta);
+  expert_scan_kernel<<<1, threads, 0, s>>>(NC, E, chunk_hist, counts, offsets, touched, group_base, tile_base,
+                                           meta);
   return cudaGetLastError();
 }
 

@@ -13,12 +13,14 @@ from gpu_util import judge, layer_from_problem, run, x_to_device
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
 
-PATHS = {"auto": moe.MOE_PATH_AUTO, "gemv": moe.MOE_PATH_GEMV}
+PATHS = {"auto": moe.MOE_PATH_AUTO, "gemv": moe.MOE_PATH_GEMV, "gemm": moe.MOE_PATH_GEMM}
 
-# small variants of each workload: same formats/routers, shapes the oracle runs in seconds
+# small variants of each workload: same formats/routers, shapes the oracle runs in seconds.
+# Token counts per expert span one to several 128-token chunks with ragged tails.
 SMALL = {
     "tiny-fp32": (1, {}),
-    "kimi-bf16-small": (2, dict(T=37, H=256, E=32, I=192)),
+    "kimi-bf16-small": (2, dict(T=37, H=256, E=32, I=256)),
+    "kimi-bf16-ragged": (2, dict(T=45, H=256, E=32, I=192)),      # I not a multiple of 128: GEMV only
     "kimi-int8-small": (3, dict(T=203, H=384, E=24, I=256)),
     "qwen3-int4-small": (4, dict(T=150, H=256, E=16, I=128)),
     "skew-masked-int8-small": (5, dict(T=301, H=256, E=40, I=128, n_active=23, bias=("skew", 0.15))),
@@ -37,6 +39,11 @@ def _clear_flags():
 def test_small_workloads(name, path):
     cid, over = SMALL[name]
     prob = synth.make_problem(cid, **over)
+    if path == "gemm" and (prob.wfmt == "f32" or prob.H % 128 or prob.I % 128):
+        with pytest.raises(moe.MoeError) as ei:
+            run(prob, PATHS[path])
+        assert ei.value.status == moe.MOE_ERR_UNSUPPORTED
+        return
     _, _, y, idx, w = run(prob, PATHS[path])
     rep = judge(prob, y, idx, w)
     assert rep["near_ties"] <= max(2, prob.T // 20)
