@@ -30,6 +30,13 @@ __device__ __forceinline__ float sigmoidf_acc(float v) { return 1.0f / (1.0f + e
 // SiLU(g) * u, the gated activation of the expert FFN
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
+// The same with CUDA's fast intrinsics (a few ulp), for outputs rounded to bf16
+// afterwards.  The exponent argument is capped so 1 + e stays below 2^126, the
+// range where __fdividef is exact to its stated error.
+__device__ __forceinline__ float silu_mul_fast(float g, float u) {
+  return __fdividef(g, 1.0f + __expf(fminf(-g, 80.0f))) * u;
+}
+
 // ---------------------------------------------------------------- flags
 
 __device__ __forceinline__ void raise_flag(uint32_t* flags, uint32_t bit) {
@@ -116,6 +123,20 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
   return v;
+}
+
+// named barrier that also ORs a predicate over the participating threads
+__device__ __forceinline__ bool named_bar_or(int id, int threads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.or.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {

@@ -2,27 +2,30 @@
 //
 // "only the 8 routed experts are computed for each token" (Qwen3-30B-A3B
 // LiteRT-LM card, Conversion Notes): after the tokens are sorted by expert,
-// every expert e owns a contiguous run of m_e rows.  Each unit of work is
-// (expert e, block of 128 weight rows, chunk of up to 128 of e's tokens) and
-// is computed swap-AB:  D[128 weight rows, N tokens] = W_blk[128, K] * X_e[N, K]^T,
-// with M = 128 fixed and N = the chunk's token count rounded up to 16, so a
-// ragged expert costs at most 15 padded columns instead of a padded 128-row tile.
+// every expert e owns a contiguous run of m_e rows.  A unit of work is
+// (expert e, block of output rows, chunk of up to `chunk` of e's tokens),
+// computed swap-AB:  D[128 weight rows, N tokens] = A[128, K] * X_e[N, K]^T,
+// M = 128 and N = the chunk's token count rounded up to 16 (<= 256), so a
+// ragged expert pays at most 15 padded columns.
 //
-//   gate/up:  h[pos, i] = SiLU(s_g D_gate[i, pos]) * (s_u D_up[i, pos])       (bf16 out)
-//   down:     Yp[pair, r] = w_pair * s_d * D_down[r, pos]                       (fp32 out)
-// Storage: bf16 weights go straight from TMA into the 128-byte-swizzled K-major
-// layout the tensor core reads; int8 (per-row scale, Kimi-Linear LiteRT-LM
-// details page, quantization bullet) is widened exactly to bf16 by dequant
-// warps and its row scale applied in the epilogue; int4 block-32 (Qwen3 card,
-// Available Artifacts table) is widened to q*s in bf16 by the dequant warps.
+//   gate/up: the 128 A rows are 64 rows of W_gate and the same 64 rows of
+//            W_up, so one accumulator holds both projections of 64 outputs:
+//            h[pos, i] = SiLU(s_g D[i, pos]) * (s_u D[64 + i, pos])  (bf16 out)
+//   down:    A = 128 rows of W_down;  Yp[pair, r] = w_pair * s_d * D[r, pos] (fp32)
+// Storage: bf16 weights go straight from TMA into the 128-byte-swizzled
+// K-major layout the tensor core reads; int8 rows (one scale per row and
+// expert -- Kimi-Linear LiteRT-LM details, quantization bullet) are widened
+// exactly to bf16 by dequant warps and scaled in the epilogue; int4 block-32
+// (Qwen3 card, Available Artifacts table) is widened to q*s in bf16.
 //
-// Roles in a persistent CTA (one per SM), all on one list of units:
-//   warp 0 lane 0   TMA producer (weights or raw quantised tiles, token tile)
-//   warp 1          TMEM allocator; lane 0 issues tcgen05.mma
-//   warps 4..7      epilogue: TMEM -> registers -> activation/scales -> global
-//   warps 8..11     dequantisation (int8 / int4 only)
-// Accumulators are double-buffered in TMEM so the epilogue of one unit
+// Roles in a persistent CTA (one per SM), all walking one list of units:
+//   warp 0 lane 0   TMA producer (weight or raw quantised tiles, token boxes)
+//   warp 1          TMEM allocator; lane 0 issues tcgen05.mma, commits stages
+//   warps 4..7      epilogue: tcgen05.ld -> activation / scales -> global
+//   warps 8..15     dequantisation (int8 / int4 only)
+// TMEM holds two accumulators of `chunk` columns, so the epilogue of one unit
 // overlaps the MMAs of the next.  Every wait is bounded (MOE_FLAG_TIMEOUT).
+// No cluster, no multicast.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -31,27 +34,38 @@
 namespace moe {
 namespace {
 
-constexpr int kBM = 128;  // weight rows per unit (MMA M)
-constexpr int kBK = 64;   // K per stage (one 128-byte swizzle row of bf16)
-constexpr int kMaxN = kTileN;  // tokens per unit
-constexpr int kTileBytes = kBM * kBK * 2;  // 16 KB bf16 tile
+constexpr int kBM = 128;                   // MMA M (weight rows per tile)
+constexpr int kBK = 64;                    // K per stage: one 128-byte swizzle row of bf16
+constexpr int kTileBytes = kBM * kBK * 2;  // A tile, 16 KB
+constexpr int kBoxRows = 32;               // token rows per TMA box
 constexpr int kMaxStages = 8;
+constexpr int kAStages = 2;                // quantised: bf16 A tiles between dequant and MMA
+constexpr int kXchgCols = 16;              // gate/up epilogue exchange: columns per step
+constexpr int kXchgBytes = 2 * kXchgCols * 64 * 4;  // double-buffered [16 cols][64 rows] fp32
+constexpr int kBarrierBytes = 1024;
+constexpr int kSmemLimit = 232448;         // 227 KB opt-in
 
 struct GemmArgs {
-  const float* s0;       // scales of W0 (int8: [E,R]; int4: [E,R,K/32])
-  const float* s1;       // scales of W1 (gate/up only)
+  const float* s0;  // scales of W0 (int8: [E,R]; int4: [E,R,K/32])
+  const float* s1;  // scales of W1 (gate/up)
   const int32_t* offsets;
   const int32_t* touched;
   const int32_t* tile_base;
   const int32_t* meta;
   const int32_t* sorted_pair;
-  const float* topk_w;   // down only
-  void* out;             // gate/up: hbuf bf16 [P, R]; down: yp fp32 [P, H]
+  const float* topk_w;  // down only
+  void* out;            // gate/up: hbuf bf16 [P, I]; down: yp fp32 [P, H]
   uint32_t* flags;
-  int R;                 // weight rows per expert (I for gate/up, H for down)
-  int K;                 // reduction length
-  int NS;                // pipeline stages
+  int R;                // weight rows per expert and matrix (I for gate/up, H for down)
+  int K;                // reduction length
+  int chunk;            // tokens per chunk (multiple of 16, <= 256)
+  int NS;               // pipeline stages
   int stage_bytes;
+  int b_off;            // B tile offset within a stage
+  int raw_off;          // raw quantised tile offset within a stage
+  int acc_stride;       // TMEM columns per M tile accumulator (power of two >= chunk)
+  int nbuf;             // accumulator buffers (2: epilogue overlaps the next unit's MMAs)
+  int tmem_cols;        // TMEM columns allocated
 };
 
 __device__ __forceinline__ void wait_or_die(uint64_t* bar, uint32_t parity, bool& dead, uint32_t* flags) {
@@ -63,10 +77,10 @@ __device__ __forceinline__ void wait_or_die(uint64_t* bar, uint32_t parity, bool
 }
 
 struct Unit {
-  int e, base, m, ib, c, n_tok, n_mma;
+  int e, base, ib, c, n_tok, n_mma;
 };
 
-// unit u -> (expert, weight-row block, token chunk); chunks fastest
+// unit u -> (expert, output-row block, token chunk); chunks fastest
 __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u, int nib, int ntouched) {
   int lo = 0, hi = ntouched - 1;
   while (lo < hi) {
@@ -77,105 +91,110 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u, int nib, i
   Unit t;
   t.e = a.touched[lo];
   t.base = a.offsets[t.e];
-  t.m = a.offsets[t.e + 1] - t.base;
-  const int nc = (t.m + kMaxN - 1) / kMaxN;
+  const int m = a.offsets[t.e + 1] - t.base;
+  const int nc = (m + a.chunk - 1) / a.chunk;
   const int r = u - a.tile_base[lo] * nib;
   t.ib = r / nc;
   t.c = r - t.ib * nc;
-  t.n_tok = min(kMaxN, t.m - t.c * kMaxN);
+  t.n_tok = min(a.chunk, m - t.c * a.chunk);
   t.n_mma = (t.n_tok + 15) & ~15;
   return t;
 }
 
-// widen one 8-element chunk of a raw quantised row to bf16 (int8: exact q;
-// int4: q * block scale, rounded to nearest even)
+// Widen one 8-element chunk of a raw quantised row to bf16.
+// int8: byte-permute (q + 128) into the low byte of the fp32 2^23 and subtract
+// 2^23 + 128 -> exact q; |q| <= 128 has <= 8 significant bits, so the top half
+// of that fp32 is the exact bf16.  int4: same for the nibble, then q * s
+// rounded to nearest even.
 template <int WF>
 __device__ __forceinline__ uint4 widen8(const uint8_t* raw_chunk, float scale) {
-  uint4 o;
+  uint32_t o[4];
   if constexpr (WF == MOE_W_INT8_ROW) {
     const uint2 w = *reinterpret_cast<const uint2*>(raw_chunk);
-    const uint32_t words[2] = {w.x, w.y};
-    uint32_t outw[4];
+    const uint32_t words[2] = {w.x ^ 0x80808080u, w.y ^ 0x80808080u};
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
+      float f[4];
 #pragma unroll
-      for (int b = 0; b < 4; b += 2) {
-        // q + 128 in the low mantissa bits of 2^23, minus (2^23 + 128): exact q
-        const float f0 = __uint_as_float(0x4B000000u | (((words[h] >> (8 * b)) & 0xFFu) ^ 0x80u)) - 8388736.0f;
-        const float f1 = __uint_as_float(0x4B000000u | (((words[h] >> (8 * b + 8)) & 0xFFu) ^ 0x80u)) - 8388736.0f;
-        // |q| <= 128 has at most 8 significant bits: the top half of the fp32 is the exact bf16
-        outw[h * 2 + b / 2] = __byte_perm(__float_as_uint(f0), __float_as_uint(f1), 0x7632);
-      }
+      for (int b = 0; b < 4; ++b)
+        f[b] = __uint_as_float(__byte_perm(words[h], 0x4B000000u, 0x7440u | b)) - 8388736.0f;
+      o[2 * h] = __byte_perm(__float_as_uint(f[0]), __float_as_uint(f[1]), 0x7632);
+      o[2 * h + 1] = __byte_perm(__float_as_uint(f[2]), __float_as_uint(f[3]), 0x7632);
     }
-    o = make_uint4(outw[0], outw[1], outw[2], outw[3]);
   } else {
     const uint32_t w = *reinterpret_cast<const uint32_t*>(raw_chunk);
-    uint32_t outw[4];
+    const uint32_t lo = (w & 0x0F0F0F0Fu) ^ 0x08080808u;         // even elements, q + 8
+    const uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;  // odd elements
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float q0 = __uint_as_float(0x4B000000u | (((w >> (8 * j)) & 0xFu) ^ 0x8u)) - 8388616.0f;
-      const float q1 = __uint_as_float(0x4B000000u | (((w >> (8 * j + 4)) & 0xFu) ^ 0x8u)) - 8388616.0f;
-      outw[j] = pack_bf16x2(q0 * scale, q1 * scale);
+      const float q0 = __uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7440u | j)) - 8388616.0f;
+      const float q1 = __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7440u | j)) - 8388616.0f;
+      o[j] = pack_bf16x2(q0 * scale, q1 * scale);
     }
-    o = make_uint4(outw[0], outw[1], outw[2], outw[3]);
   }
-  return o;
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-template <int MODE, int WF>
-struct Layout {
-  static constexpr int NMAT = MODE == 0 ? 2 : 1;
+template <int MODE, int WF, int MT>
+struct Traits {
   static constexpr bool kQuant = WF != MOE_W_BF16;
-  static constexpr int kRawBytes = WF == MOE_W_INT8_ROW ? kBM * kBK : (WF == MOE_W_INT4_B32 ? kBM * kBK / 2 : 0);
-  // stage: [A_0 .. A_{NMAT-1}] (bf16 16 KB each) [B tokens 16 KB] [raw_0 .. raw_{NMAT-1}]
-  static constexpr int kA = 0;
-  static constexpr int kB = NMAT * kTileBytes;
-  static constexpr int kRaw = kB + kMaxN * kBK * 2;
-  static constexpr int kStage = kRaw + NMAT * kRawBytes;
-  static constexpr int kThreads = kQuant ? 384 : 256;
-  static constexpr int kAccCols = NMAT * kMaxN;  // TMEM columns per accumulator buffer
-  static constexpr int kTmemCols = 2 * kAccCols; // double-buffered (256 or 512)
+  static constexpr int kTileRows = MODE == 0 ? 64 : 128;  // output rows per M tile
+  static constexpr int kRows = kTileRows * MT;            // output rows per unit
+  static constexpr int kRawTile = WF == MOE_W_INT8_ROW ? kBM * kBK : (WF == MOE_W_INT4_B32 ? kBM * kBK / 2 : 0);
+  static constexpr int kRawPitch = WF == MOE_W_INT8_ROW ? kBK : kBK / 2;  // bytes per raw row
+  static constexpr int kEpiWarps = 4 * MT;                // one 4-warp group per M tile
+  static constexpr int kDequantWarps = kQuant ? 8 : 0;
+  static constexpr int kDequant0 = 4 + kEpiWarps;         // first dequant warp
+  static constexpr int kThreads = 32 * (4 + kEpiWarps + kDequantWarps);
+  // per group: gate/up exchange of up values between TMEM quadrants (8 KB);
+  // down: the unit's pair ids and routing weights (2 KB)
+  static constexpr int kGroupXchg = MODE == 0 ? kXchgBytes : 2 * 256 * 4;
+  static constexpr int kXchg = (MT * kGroupXchg + 1023) / 1024 * 1024;
 };
 
-template <int MODE, int WF>
-__global__ void __launch_bounds__(Layout<MODE, WF>::kThreads, 1)
+template <int MODE, int WF, int MT>
+__global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
                    const __grid_constant__ CUtensorMap tm_b, const GemmArgs a) {
-  using L = Layout<MODE, WF>;
-  constexpr int NMAT = L::NMAT;
+  using Tr = Traits<MODE, WF, MT>;
   extern __shared__ uint8_t smem_raw[];
-  // 1024-byte aligned base for the swizzled tiles
   const uint32_t raw_base = smem_u32(smem_raw);
-  const uint32_t pad = ((raw_base + 1023u) & ~1023u) - raw_base;
-  uint8_t* smem = smem_raw + pad;
-  uint8_t* stages = smem + 1024;  // first 1 KB: barriers and the TMEM address
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem);       // TMA landed (bf16: A+B; quant: raw+B)
-  uint64_t* ready = full + kMaxStages;                      // quant: bf16 A written by dequant warps
-  uint64_t* empty = ready + kMaxStages;                     // MMA finished reading the stage
-  uint64_t* acc_full = empty + kMaxStages;                  // [2] accumulator complete
-  uint64_t* acc_empty = acc_full + 2;                       // [2] epilogue drained the accumulator
-  uint64_t* mma_done = acc_empty + 2;                       // final completion of all MMAs
+  uint8_t* smem = smem_raw + (((raw_base + 1023u) & ~1023u) - raw_base);  // 1024-aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);  // TMA landed (A or raw, and B)
+  uint64_t* empty = full + kMaxStages;                 // MMAs finished reading the stage
+  uint64_t* ready = empty + kMaxStages;                // [kAStages] quantised: bf16 A written
+  uint64_t* a_empty = ready + kAStages;                // [kAStages] quantised: MMAs done with bf16 A
+  uint64_t* acc_full = a_empty + kAStages;             // [2]
+  uint64_t* acc_empty = acc_full + 2;                  // [2]
+  uint64_t* mma_done = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  float* xchg = reinterpret_cast<float*>(smem + kBarrierBytes);
+  uint8_t* a_ring = smem + kBarrierBytes + Tr::kXchg;  // quantised: kAStages x MT bf16 A tiles
+  uint8_t* stages = a_ring + (Tr::kQuant ? kAStages * MT * kTileBytes : 0);
 
   const int w = warp_id(), lane = lane_id();
-  const int NS = a.NS;
+  const int NS = a.NS, nbuf = a.nbuf;
+  const uint32_t buf_cols = (uint32_t)(MT * a.acc_stride);
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&ready[i], 4);
       mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < kAStages; ++i) {
+      mbar_init(&ready[i], Tr::kDequantWarps > 0 ? Tr::kDequantWarps : 1);
+      mbar_init(&a_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4);
+      mbar_init(&acc_empty[i], Tr::kEpiWarps);
     }
     mbar_init(mma_done, 1);
     fence_mbar_init();
   }
-  if (w == 1) tmem_alloc(tmem_slot, L::kTmemCols);
+  if (w == 1) tmem_alloc(tmem_slot, (uint32_t)a.tmem_cols);
   if (threadIdx.x == 32) {
     prefetch_tmap(&tm_w0);
-    if (NMAT == 2) prefetch_tmap(&tm_w1);
+    if (MODE == 0) prefetch_tmap(&tm_w1);
     prefetch_tmap(&tm_b);
   }
   tc_fence_before();
@@ -184,70 +203,80 @@ __global__ void __launch_bounds__(Layout<MODE, WF>::kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int ntouched = a.meta[0];
-  const int nib = a.R / kBM;
+  const int nib = a.R / Tr::kRows;
   const int total = ntouched > 0 ? a.meta[3] * nib : 0;
   const int nk = a.K / kBK;
 
   if (w == 0) {
-    // ---------------------------------------------------------------- TMA producer
+    // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       bool dead = false;
       uint32_t it = 0;
+      const uint32_t abytes = MT * (Tr::kQuant ? Tr::kRawTile : kTileBytes);
       for (int u = blockIdx.x; u < total; u += gridDim.x) {
         const Unit t = decode_unit(a, u, nib, ntouched);
-        const int nbox = (t.n_tok + 31) / 32;
-        const int brow = t.base + t.c * kMaxN;
-        const int wrow = t.e * a.R + t.ib * kBM;
+        const int nbox = (t.n_tok + kBoxRows - 1) / kBoxRows;
+        const int brow = t.base + t.c * a.chunk;
+        const int wrow0 = t.e * a.R + t.ib * Tr::kRows;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % NS;
           wait_or_die(&empty[s], ((it / NS) & 1u) ^ 1u, dead, a.flags);
           if (dead) continue;
           uint8_t* st = stages + (size_t)s * a.stage_bytes;
-          const uint32_t wbytes = L::kQuant ? L::kRawBytes : kTileBytes;
-          mbar_arrive_expect_tx(&full[s], NMAT * wbytes + nbox * 32 * kBK * 2);
-          // weights: bf16 straight into the swizzled A tile; quantised into the raw area
-          const int wcol = WF == MOE_W_INT4_B32 ? kb * kBK / 2 : kb * kBK;  // int4: bytes
-          tma_load_2d(L::kQuant ? st + L::kRaw : st + L::kA, &tm_w0, wcol, wrow, &full[s]);
-          if (NMAT == 2)
-            tma_load_2d(L::kQuant ? st + L::kRaw + L::kRawBytes : st + L::kA + kTileBytes, &tm_w1, wcol, wrow,
-                        &full[s]);
-          for (int j = 0; j < nbox; ++j) tma_load_2d(st + L::kB + j * 32 * kBK * 2, &tm_b, kb * kBK, brow + 32 * j, &full[s]);
+          mbar_arrive_expect_tx(&full[s], abytes + nbox * kBoxRows * kBK * 2);
+          const int wcol = WF == MOE_W_INT4_B32 ? kb * (kBK / 2) : kb * kBK;  // int4 maps count bytes
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            uint8_t* adst = Tr::kQuant ? st + a.raw_off + mt * Tr::kRawTile : st + mt * kTileBytes;
+            const int wrow = wrow0 + mt * Tr::kTileRows;
+            if (MODE == 0) {
+              const int half = Tr::kQuant ? 64 * Tr::kRawPitch : kTileBytes / 2;
+              tma_load_2d(adst, &tm_w0, wcol, wrow, &full[s]);         // 64 gate rows
+              tma_load_2d(adst + half, &tm_w1, wcol, wrow, &full[s]);  // the same 64 up rows
+            } else {
+              tma_load_2d(adst, &tm_w0, wcol, wrow, &full[s]);         // 128 down rows
+            }
+          }
+          for (int j = 0; j < nbox; ++j)
+            tma_load_2d(st + a.b_off + j * kBoxRows * kBK * 2, &tm_b, kb * kBK, brow + kBoxRows * j, &full[s]);
         }
       }
-      // stay until the last stages' copies have landed
       const uint32_t first = it > (uint32_t)NS ? it - NS : 0u;
       for (uint32_t j = first; j < it && !dead; ++j) wait_or_die(&full[j % NS], (j / NS) & 1u, dead, a.flags);
     }
   } else if (w == 1) {
-    // ---------------------------------------------------------------- MMA issuer
+    // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool dead = false;
       uint32_t it = 0, local = 0;
       const uint32_t stage0 = smem_u32(stages);
+      const uint32_t a_ring0 = smem_u32(a_ring);
       for (int u = blockIdx.x; u < total; u += gridDim.x, ++local) {
         const Unit t = decode_unit(a, u, nib, ntouched);
-        const uint32_t buf = local & 1u;
-        wait_or_die(&acc_empty[buf], ((local >> 1) & 1u) ^ 1u, dead, a.flags);
+        const uint32_t buf = local % nbuf;
+        wait_or_die(&acc_empty[buf], ((local / nbuf) & 1u) ^ 1u, dead, a.flags);
         tc_fence_after();
         const uint32_t idesc = umma_idesc_bf16(kBM, t.n_mma);
-        const uint32_t d0 = tmem_base + buf * L::kAccCols;
+        const uint32_t d = tmem_base + buf * buf_cols;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % NS;
-          const uint32_t par = (it / NS) & 1u;
-          wait_or_die(L::kQuant ? &ready[s] : &full[s], par, dead, a.flags);
-          if (L::kQuant) wait_or_die(&full[s], par, dead, a.flags);  // token tile landed too
+          const int ja = it % kAStages;
+          if (Tr::kQuant) wait_or_die(&ready[ja], (it / kAStages) & 1u, dead, a.flags);
+          wait_or_die(&full[s], (it / NS) & 1u, dead, a.flags);
           if (dead) continue;
           tc_fence_after();
-          const uint32_t sa = stage0 + s * a.stage_bytes;
+          const uint32_t sb = stage0 + s * a.stage_bytes;
+          const uint32_t sa = Tr::kQuant ? a_ring0 + ja * (MT * kTileBytes) : sb;
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
-            const uint64_t bdesc = umma_desc_sw128(sa + L::kB + k * 32);
+            const uint64_t bdesc = umma_desc_sw128(sb + a.b_off + k * 32);
 #pragma unroll
-            for (int mtx = 0; mtx < NMAT; ++mtx)
-              umma_bf16(d0 + mtx * kMaxN, umma_desc_sw128(sa + L::kA + mtx * kTileBytes + k * 32), bdesc, idesc,
+            for (int mt = 0; mt < MT; ++mt)
+              umma_bf16(d + mt * a.acc_stride, umma_desc_sw128(sa + mt * kTileBytes + k * 32), bdesc, idesc,
                         (kb | k) != 0);
           }
           umma_commit(&empty[s]);
+          if (Tr::kQuant) umma_commit(&a_empty[ja]);
         }
         if (!dead) umma_commit(&acc_full[buf]);
       }
@@ -256,55 +285,75 @@ __global__ void __launch_bounds__(Layout<MODE, WF>::kThreads, 1)
         wait_or_die(mma_done, 0, dead, a.flags);
       }
     }
-  } else if (w >= 4 && w < 8) {
-    // ---------------------------------------------------------------- epilogue
-    const int q = w - 4;                // TMEM lanes 32q .. 32q+31
-    const int row_in_blk = q * 32 + lane;
+  } else if (w >= 4 && w < 4 + Tr::kEpiWarps) {
+    // ------------------------------------------------------------------ epilogue
+    const int grp = (w - 4) >> 2;  // M tile drained by this 4-warp group
+    const int q = w & 3;           // TMEM lanes 32q .. 32q+31
+    const int bar_x = 1 + 2 * grp, bar_v = 2 + 2 * grp;
+    float* gx = xchg + grp * (Tr::kGroupXchg / 4);
     bool dead = false;
-    uint32_t local = 0;
+    uint32_t local = 0, xc = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x, ++local) {
       const Unit t = decode_unit(a, u, nib, ntouched);
-      const uint32_t buf = local & 1u;
-      // one lane waits, the warp follows its verdict (the TMEM loads below are warp-collective)
-      if (lane == 0) wait_or_die(&acc_full[buf], (local >> 1) & 1u, dead, a.flags);
-      dead = __shfl_sync(0xFFFFFFFFu, dead ? 1 : 0, 0) != 0;
-      __syncwarp();
+      const uint32_t buf = local % nbuf;
+      if (lane == 0) wait_or_die(&acc_full[buf], (local / nbuf) & 1u, dead, a.flags);
+      // the group's four warps agree on the verdict (their loops hold named barriers)
+      dead = named_bar_or(bar_v, 128, dead);
       tc_fence_after();
+      const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * buf_cols + grp * a.acc_stride;
+      const int pos0 = t.base + t.c * a.chunk;
       if (!dead) {
-        const int row = t.ib * kBM + row_in_blk;
-        const size_t grow = (size_t)t.e * a.R + row;
-        const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * L::kAccCols;
-        const int pos0 = t.base + t.c * kMaxN;
         if (MODE == 0) {
+          // lanes 0..63 hold gate rows, 64..127 the matching up rows: up warps hand
+          // their values to the gate warps through a double-buffered exchange
+          const int r64 = (q & 1) * 32 + lane;
+          const int row = t.ib * Tr::kRows + grp * 64 + r64;
+          const size_t grow = (size_t)t.e * a.R + row;
           const float sg = WF == MOE_W_INT8_ROW ? a.s0[grow] : 1.f;
           const float su = WF == MOE_W_INT8_ROW ? a.s1[grow] : 1.f;
-          uint16_t* h = static_cast<uint16_t*>(a.out);
-          for (int n0 = 0; n0 < t.n_tok; n0 += 16) {
-            uint32_t g[16], v[16];
-            tmem_ld16(tacc + n0, g);
-            tmem_ld16(tacc + kMaxN + n0, v);
+          uint16_t* hout = static_cast<uint16_t*>(a.out);
+          for (int n0 = 0; n0 < t.n_tok; n0 += kXchgCols, ++xc) {
+            float* xb = gx + (xc & 1u) * (kXchgCols * 64);
+            uint32_t v[16];
+            tmem_ld16(tacc + n0, v);
             tmem_ld_wait();
+            if (q >= 2) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              if (n0 + j < t.n_tok) {
-                const float hv = silu_mul(__uint_as_float(g[j]) * sg, __uint_as_float(v[j]) * su);
-                h[(size_t)(pos0 + n0 + j) * a.R + row] = f32_to_bf16(hv);
+              for (int j = 0; j < 16; ++j) xb[j * 64 + r64] = __uint_as_float(v[j]);
+            }
+            named_bar_sync(bar_x, 128);
+            if (q < 2) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                if (n0 + j < t.n_tok) {
+                  const float hv = silu_mul_fast(__uint_as_float(v[j]) * sg, xb[j * 64 + r64] * su);
+                  hout[(size_t)(pos0 + n0 + j) * a.R + row] = f32_to_bf16(hv);
+                }
               }
             }
           }
         } else {
-          const float sd = WF == MOE_W_INT8_ROW ? a.s0[grow] : 1.f;
+          // stage the unit's pair ids and routing weights (one round trip for all columns)
+          int32_t* s_pair = reinterpret_cast<int32_t*>(gx);
+          float* s_w = gx + 256;
+          const int et = q * 32 + lane;
+          for (int n = et; n < t.n_tok; n += 128) {
+            const int pair = a.sorted_pair[pos0 + n];
+            s_pair[n] = pair;
+            s_w[n] = a.topk_w[pair];
+          }
+          named_bar_sync(bar_x, 128);
+          const int row = t.ib * Tr::kRows + grp * 128 + et;
+          const float sd = WF == MOE_W_INT8_ROW ? a.s0[(size_t)t.e * a.R + row] : 1.f;
           float* yp = static_cast<float*>(a.out);
           for (int n0 = 0; n0 < t.n_tok; n0 += 16) {
-            uint32_t d[16];
-            tmem_ld16(tacc + n0, d);
+            uint32_t v[16];
+            tmem_ld16(tacc + n0, v);
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              if (n0 + j < t.n_tok) {
-                const int pair = a.sorted_pair[pos0 + n0 + j];
-                yp[(size_t)pair * a.R + row] = a.topk_w[pair] * sd * __uint_as_float(d[j]);
-              }
+              if (n0 + j < t.n_tok)
+                yp[(size_t)s_pair[n0 + j] * a.R + row] = s_w[n0 + j] * sd * __uint_as_float(v[j]);
             }
           }
         }
@@ -313,38 +362,56 @@ __global__ void __launch_bounds__(Layout<MODE, WF>::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
-  } else if (L::kQuant && w >= 8) {
-    // ---------------------------------------------------------------- dequantisation
-    const int ct = threadIdx.x - 256;  // 0..127
+  } else if (Tr::kQuant && w >= Tr::kDequant0) {
+    // ------------------------------------------------------------------ dequantisation
+    // thread ct widens chunks (r, c8): r = ct/8 + kRowStep*j over the unit's MT*128
+    // weight rows, c8 = ct%8 -- 8 elements each
+    constexpr int kDT = 32 * (Tr::kDequantWarps > 0 ? Tr::kDequantWarps : 1);
+    constexpr int kRowStep = kDT / 8;
+    constexpr int kPer = MT * kBM / kRowStep;  // chunks per thread per K step
+    const int ct = threadIdx.x - 32 * Tr::kDequant0;
+    const int c8 = ct & 7, r0 = ct >> 3;
     bool dead = false;
     uint32_t it = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
       const Unit t = decode_unit(a, u, nib, ntouched);
-      for (int kb = 0; kb < nk; ++kb, ++it) {
-        const int s = it % NS;
-        wait_or_die(&full[s], (it / NS) & 1u, dead, a.flags);
-        if (!dead) {
-          uint8_t* st = stages + (size_t)s * a.stage_bytes;
+      // int4: block scales of this thread's rows, one K step ahead
+      const float* srow[kPer];
+      float sc_next[kPer];
 #pragma unroll
-          for (int mtx = 0; mtx < NMAT; ++mtx) {
-            const uint8_t* raw = st + L::kRaw + mtx * L::kRawBytes;
-            uint8_t* A = st + L::kA + mtx * kTileBytes;
-            const float* S = mtx ? a.s1 : a.s0;
-#pragma unroll 2
-            for (int i = ct; i < kBM * 8; i += 128) {
-              const int r = i >> 3, c8 = i & 7;
-              float sc = 1.f;
-              if (WF == MOE_W_INT4_B32)
-                sc = __ldg(S + ((size_t)t.e * a.R + t.ib * kBM + r) * (a.K / 32) + kb * 2 + (c8 >> 2));
-              const int rb = WF == MOE_W_INT8_ROW ? r * kBK + c8 * 8 : r * (kBK / 2) + c8 * 4;
-              const uint4 v = widen8<WF>(raw + rb, sc);
-              *reinterpret_cast<uint4*>(A + r * 128 + ((c8 ^ (r & 7)) << 4)) = v;
-            }
+      for (int j = 0; j < kPer; ++j) {
+        const int r = r0 + kRowStep * j;  // row within the unit's MT*128 A rows
+        const int mt = r >> 7, rr = r & 127;
+        const float* S = (MODE == 0 && rr >= 64) ? a.s1 : a.s0;
+        const int wr = t.ib * Tr::kRows + mt * Tr::kTileRows + (MODE == 0 ? (rr & 63) : rr);
+        srow[j] = S + ((size_t)t.e * a.R + wr) * (a.K / 32) + (c8 >> 2);
+        sc_next[j] = WF == MOE_W_INT4_B32 ? __ldg(srow[j]) : 1.f;
+      }
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        float sc[kPer];
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+          sc[j] = sc_next[j];
+          if (WF == MOE_W_INT4_B32 && kb + 1 < nk) sc_next[j] = __ldg(srow[j] + (kb + 1) * 2);
+        }
+        const int s = it % NS;
+        const int ja = it % kAStages;
+        wait_or_die(&full[s], (it / NS) & 1u, dead, a.flags);
+        wait_or_die(&a_empty[ja], ((it / kAStages) & 1u) ^ 1u, dead, a.flags);
+        if (!dead) {
+          const uint8_t* raw = stages + (size_t)s * a.stage_bytes + a.raw_off;
+          uint8_t* A = a_ring + ja * (MT * kTileBytes);
+#pragma unroll
+          for (int j = 0; j < kPer; ++j) {
+            const int r = r0 + kRowStep * j;
+            const int mt = r >> 7, rr = r & 127;
+            const uint4 v = widen8<WF>(raw + mt * Tr::kRawTile + rr * Tr::kRawPitch + c8 * (Tr::kRawPitch / 8), sc[j]);
+            *reinterpret_cast<uint4*>(A + mt * kTileBytes + rr * 128 + ((c8 ^ (rr & 7)) << 4)) = v;
           }
           fence_proxy_async_smem();
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ready[s]);
+        if (lane == 0) mbar_arrive(&ready[ja]);
       }
     }
   }
@@ -353,7 +420,7 @@ __global__ void __launch_bounds__(Layout<MODE, WF>::kThreads, 1)
   __syncthreads();
   if (w == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, L::kTmemCols);
+    tmem_dealloc(tmem_base, (uint32_t)a.tmem_cols);
   }
 }
 
@@ -389,42 +456,68 @@ cudaError_t make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, i
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t weight_map(CUtensorMap* m, const void* W, int wfmt, int E, int R, int K) {
+cudaError_t weight_map(CUtensorMap* m, const void* W, int wfmt, int E, int R, int K, int box_rows) {
   const uint64_t rows = (uint64_t)E * R;
   if (wfmt == MOE_W_BF16)
-    return make_map(m, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, rows, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B);
+    return make_map(m, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, rows, kBK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
   if (wfmt == MOE_W_INT8_ROW)
-    return make_map(m, W, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, rows, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_NONE);
-  return make_map(m, W, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, rows, kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_NONE);
+    return make_map(m, W, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, rows, kBK, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
+  return make_map(m, W, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, rows, kBK / 2, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-template <int MODE, int WF>
+uint32_t pow2_at_least(uint32_t v) {
+  uint32_t p = 32;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+template <int MODE, int WF, int MT>
 cudaError_t launch_gemm(const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb, GemmArgs a,
                         int num_sms, cudaStream_t s) {
-  using L = Layout<MODE, WF>;
-  a.stage_bytes = L::kStage;
-  const int budget = 232448 - 2048;  // opt-in limit minus barriers and alignment slack
-  a.NS = budget / L::kStage;
+  using Tr = Traits<MODE, WF, MT>;
+  // stage: bf16 weights [A: MT x 16 KB][B]; quantised [B][raw: MT tiles] (their bf16 A lives
+  // in the A ring).  Token boxes are kBoxRows tall: B holds the chunk rounded up to whole boxes.
+  const int b_rows = (a.chunk + kBoxRows - 1) / kBoxRows * kBoxRows;
+  a.b_off = Tr::kQuant ? 0 : MT * kTileBytes;
+  a.raw_off = a.b_off + b_rows * kBK * 2;
+  a.stage_bytes = a.raw_off + MT * Tr::kRawTile;  // multiple of 1024 (4 KB boxes, 16/8/4 KB tiles)
+  a.acc_stride = (int)pow2_at_least((uint32_t)a.chunk);
+  a.nbuf = 2 * MT * a.acc_stride <= 512 ? 2 : 1;
+  a.tmem_cols = a.nbuf * MT * a.acc_stride;
+  const int fixed = 1024 + kBarrierBytes + Tr::kXchg + (Tr::kQuant ? kAStages * MT * kTileBytes : 0);
+  a.NS = (kSmemLimit - fixed) / a.stage_bytes;
   if (a.NS > kMaxStages) a.NS = kMaxStages;
-  const size_t smem = 2048 + (size_t)a.NS * L::kStage;
-  auto kern = gemm_tc_kernel<MODE, WF>;
+  if (a.NS < 2) return cudaErrorInvalidConfiguration;
+  const size_t smem = (size_t)fixed + (size_t)a.NS * a.stage_bytes;
+  auto kern = gemm_tc_kernel<MODE, WF, MT>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  kern<<<num_sms, L::kThreads, smem, s>>>(m0, m1, mb, a);
+  kern<<<num_sms, Tr::kThreads, smem, s>>>(m0, m1, mb, a);
   return cudaGetLastError();
 }
 
+// two M tiles per unit (B reused across 256 weight rows) once chunks are large
+// enough for the tensor core to be the bottleneck; one tile for small batches,
+// where finer units balance the weight stream across SMs
 template <int MODE>
 cudaError_t launch_by_format(int wfmt, const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb,
                              const GemmArgs& a, int num_sms, cudaStream_t s) {
+  const int tile_rows = MODE == 0 ? 64 : 128;
+  const bool two = a.chunk >= 128 && a.R % (2 * tile_rows) == 0;
   switch (wfmt) {
-    case MOE_W_BF16: return launch_gemm<MODE, MOE_W_BF16>(m0, m1, mb, a, num_sms, s);
-    case MOE_W_INT8_ROW: return launch_gemm<MODE, MOE_W_INT8_ROW>(m0, m1, mb, a, num_sms, s);
-    default: return launch_gemm<MODE, MOE_W_INT4_B32>(m0, m1, mb, a, num_sms, s);
+    case MOE_W_BF16:
+      return two ? launch_gemm<MODE, MOE_W_BF16, 2>(m0, m1, mb, a, num_sms, s)
+                 : launch_gemm<MODE, MOE_W_BF16, 1>(m0, m1, mb, a, num_sms, s);
+    case MOE_W_INT8_ROW:
+      return two ? launch_gemm<MODE, MOE_W_INT8_ROW, 2>(m0, m1, mb, a, num_sms, s)
+                 : launch_gemm<MODE, MOE_W_INT8_ROW, 1>(m0, m1, mb, a, num_sms, s);
+    default:
+      return two ? launch_gemm<MODE, MOE_W_INT4_B32, 2>(m0, m1, mb, a, num_sms, s)
+                 : launch_gemm<MODE, MOE_W_INT4_B32, 1>(m0, m1, mb, a, num_sms, s);
   }
 }
 
-GemmArgs common(const Workspace& ws, uint32_t* flags) {
+GemmArgs common(const Workspace& ws, int chunk, uint32_t* flags) {
   GemmArgs a{};
   a.offsets = ws.offsets;
   a.touched = ws.touched;
@@ -432,6 +525,7 @@ GemmArgs common(const Workspace& ws, uint32_t* flags) {
   a.meta = ws.meta;
   a.sorted_pair = ws.sorted_pair;
   a.flags = flags;
+  a.chunk = chunk;
   return a;
 }
 
@@ -450,8 +544,9 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
 
 }  // namespace
 
+// gate/up tiles 64 output rows (K = H); down tiles 128 rows of H (K = I)
 bool gemm_tc_supported(const moe_desc& d) {
-  return d.xfmt == MOE_X_BF16 && d.wfmt != MOE_W_F32 && d.H % kBM == 0 && d.I % kBM == 0 && encode_fn() != nullptr;
+  return d.xfmt == MOE_X_BF16 && d.wfmt != MOE_W_F32 && d.H % 128 == 0 && d.I % 64 == 0 && encode_fn() != nullptr;
 }
 
 cudaError_t launch_gather_rows(const moe_desc& d, const void* x, const Workspace& ws, int P, int num_sms,
@@ -465,15 +560,16 @@ cudaError_t launch_gather_rows(const moe_desc& d, const void* x, const Workspace
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_gateup(const moe_desc& d, const Workspace& ws, int P, int num_sms, uint32_t* flags,
-                               cudaStream_t s) {
+cudaError_t launch_gemm_gateup(const moe_desc& d, const Workspace& ws, int P, int chunk, int num_sms,
+                               uint32_t* flags, cudaStream_t s) {
   CUtensorMap mg, mu, mb;
-  cudaError_t e = weight_map(&mg, d.W_gate, d.wfmt, d.E, d.I, d.H);
-  if (e == cudaSuccess) e = weight_map(&mu, d.W_up, d.wfmt, d.E, d.I, d.H);
+  cudaError_t e = weight_map(&mg, d.W_gate, d.wfmt, d.E, d.I, d.H, 64);
+  if (e == cudaSuccess) e = weight_map(&mu, d.W_up, d.wfmt, d.E, d.I, d.H, 64);
   if (e == cudaSuccess)
-    e = make_map(&mb, ws.xs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.H, (uint64_t)P, kBK, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+    e = make_map(&mb, ws.xs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.H, (uint64_t)P, kBK, kBoxRows,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
-  GemmArgs a = common(ws, flags);
+  GemmArgs a = common(ws, chunk, flags);
   a.s0 = d.s_gate;
   a.s1 = d.s_up;
   a.out = ws.hbuf;
@@ -482,15 +578,15 @@ cudaError_t launch_gemm_gateup(const moe_desc& d, const Workspace& ws, int P, in
   return launch_by_format<0>(d.wfmt, mg, mu, mb, a, num_sms, s);
 }
 
-cudaError_t launch_gemm_down(const moe_desc& d, const float* topk_w, const Workspace& ws, int P, int num_sms,
-                             uint32_t* flags, cudaStream_t s) {
+cudaError_t launch_gemm_down(const moe_desc& d, const float* topk_w, const Workspace& ws, int P, int chunk,
+                             int num_sms, uint32_t* flags, cudaStream_t s) {
   CUtensorMap md, mb;
-  cudaError_t e = weight_map(&md, d.W_down, d.wfmt, d.E, d.H, d.I);
+  cudaError_t e = weight_map(&md, d.W_down, d.wfmt, d.E, d.H, d.I, 128);
   if (e == cudaSuccess)
-    e = make_map(&mb, ws.hbuf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.I, (uint64_t)P, kBK, 32,
+    e = make_map(&mb, ws.hbuf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.I, (uint64_t)P, kBK, kBoxRows,
                  CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
-  GemmArgs a = common(ws, flags);
+  GemmArgs a = common(ws, chunk, flags);
   a.s0 = d.s_down;
   a.topk_w = topk_w;
   a.out = ws.yp;

@@ -16,9 +16,15 @@ constexpr int kPairChunk = 1024;
 // many (every group re-reads the expert's weights, mostly from L2).
 constexpr int kGemvGroup = 4;
 
-// The tensor-core path computes an expert's tokens in chunks of this many
-// (the N of one MMA tile).
-constexpr int kTileN = 128;
+// The tensor-core path computes an expert's tokens in chunks of at most
+// kMaxTileN (the N of one MMA tile).  A batch of T tokens routes at most T
+// of them to one expert, so small batches use smaller chunks (and smaller
+// pipeline stages): chunk = min(kMaxTileN, T rounded up to 16).
+constexpr int kMaxTileN = 256;
+inline int chunk_tokens(int T) {
+  const int t = ((T > 0 ? T : 1) + 15) / 16 * 16;
+  return t < kMaxTileN ? t : kMaxTileN;
+}
 
 // Split of the router's reduction over H into S partial sums (summed in a
 // fixed order by the top-k kernel).  Depends on T only, so a masked layer and
@@ -35,7 +41,7 @@ struct Workspace {
   int32_t* meta;      // [16] device scalars: [0] touched experts, [1] valid pairs, [2] token groups,
                       //       [3] token chunks
   int32_t* group_base;  // [E + 1] first token group of each touched expert (touched order)
-  int32_t* tile_base;   // [E + 1] first token chunk (kTileN) of each touched expert
+  int32_t* tile_base;   // [E + 1] first token chunk of each touched expert
   int32_t* sorted_pair;  // [P] pair id (t * k + slot) at each sorted position
   void* hbuf;         // [P, I] activations between the two projections (bf16, or fp32 for fp32 weights)
   float* yp;          // [P, H] per-pair expert outputs times routing weight, indexed by pair id
@@ -60,8 +66,8 @@ cudaError_t launch_router_topk(const moe_desc& d, const float* partial, int S, i
 cudaError_t launch_pair_histogram(const int32_t* idx, int P, int E, int32_t* chunk_hist,
                                   uint32_t* flags, cudaStream_t s);
 cudaError_t launch_expert_scan(int NC, int E, int32_t* chunk_hist, int32_t* counts, int32_t* offsets,
-                               int32_t* touched, int32_t* group_base, int32_t* tile_base, int32_t* meta,
-                               cudaStream_t s);
+                               int32_t* touched, int32_t* group_base, int32_t* tile_base, int chunk,
+                               int32_t* meta, cudaStream_t s);
 cudaError_t launch_pair_scatter(const int32_t* idx, int P, int E, const int32_t* chunk_hist,
                                 int32_t* sorted_pair, cudaStream_t s);
 cudaError_t launch_gemv_gateup(const moe_desc& d, const void* x, int k, const Workspace& ws,
@@ -71,10 +77,10 @@ cudaError_t launch_gemv_down(const moe_desc& d, const float* topk_w, int k, cons
 bool gemm_tc_supported(const moe_desc& d);
 cudaError_t launch_gather_rows(const moe_desc& d, const void* x, const Workspace& ws, int P, int num_sms,
                                cudaStream_t s);
-cudaError_t launch_gemm_gateup(const moe_desc& d, const Workspace& ws, int P, int num_sms, uint32_t* flags,
-                               cudaStream_t s);
-cudaError_t launch_gemm_down(const moe_desc& d, const float* topk_w, const Workspace& ws, int P, int num_sms,
-                             uint32_t* flags, cudaStream_t s);
+cudaError_t launch_gemm_gateup(const moe_desc& d, const Workspace& ws, int P, int chunk, int num_sms,
+                               uint32_t* flags, cudaStream_t s);
+cudaError_t launch_gemm_down(const moe_desc& d, const float* topk_w, const Workspace& ws, int P, int chunk,
+                             int num_sms, uint32_t* flags, cudaStream_t s);
 cudaError_t launch_combine(const moe_desc& d, const int32_t* idx, int T, const float* yp, void* y,
                            cudaStream_t s);
 

@@ -298,12 +298,13 @@ extern "C" moe_status moe_forward(const moe_desc* d, const void* x, int32_t T, c
   MOE_LAUNCH("pair_histogram", stream, launch_pair_histogram(topk_idx, P, d->E, ws.chunk_hist, dev->flags, stream));
   MOE_LAUNCH("expert_scan", stream,
              launch_expert_scan(NC, d->E, ws.chunk_hist, ws.counts, ws.offsets, ws.touched, ws.group_base,
-                                ws.tile_base, ws.meta, stream));
+                                ws.tile_base, chunk_tokens(T), ws.meta, stream));
   MOE_LAUNCH("pair_scatter", stream, launch_pair_scatter(topk_idx, P, d->E, ws.chunk_hist, ws.sorted_pair, stream));
   if (path == MOE_PATH_GEMM) {
     MOE_LAUNCH("gather_rows", stream, launch_gather_rows(*d, x, ws, P, dev->num_sms, stream));
-    MOE_LAUNCH("gemm_gateup", stream, launch_gemm_gateup(*d, ws, P, dev->num_sms, dev->flags, stream));
-    MOE_LAUNCH("gemm_down", stream, launch_gemm_down(*d, topk_w, ws, P, dev->num_sms, dev->flags, stream));
+    const int chunk = chunk_tokens(T);
+    MOE_LAUNCH("gemm_gateup", stream, launch_gemm_gateup(*d, ws, P, chunk, dev->num_sms, dev->flags, stream));
+    MOE_LAUNCH("gemm_down", stream, launch_gemm_down(*d, topk_w, ws, P, chunk, dev->num_sms, dev->flags, stream));
   } else {
     MOE_LAUNCH("gemv_gateup", stream, launch_gemv_gateup(*d, x, d->k, ws, dev->num_sms, dev->flags, stream));
     MOE_LAUNCH("gemv_down", stream, launch_gemv_down(*d, topk_w, d->k, ws, dev->num_sms, dev->flags, stream));

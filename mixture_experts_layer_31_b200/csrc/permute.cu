@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(1024) expert_scan_kernel(int NC, int E, int32_
                                                            int32_t* __restrict__ offsets,
                                                            int32_t* __restrict__ touched,
                                                            int32_t* __restrict__ group_base,
-                                                           int32_t* __restrict__ tile_base,
+                                                           int32_t* __restrict__ tile_base, int chunk,
                                                            int32_t* __restrict__ meta) {
   __shared__ int warp_sums[32];
   const int e = threadIdx.x;
@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(1024) expert_scan_kernel(int NC, int E, int32_
   const int gpos = block_exclusive_scan(groups, warp_sums, &ngroups);
   if (e < E && running > 0) group_base[tpos] = gpos;
   // token chunks of the tensor-core path, same order
-  const int chunks = (e < E) ? (running + kTileN - 1) / kTileN : 0;
+  const int chunks = (e < E) ? (running + chunk - 1) / chunk : 0;
   int nchunks;
   const int cpos = block_exclusive_scan(chunks, warp_sums, &nchunks);
   if (e < E && running > 0) tile_base[tpos] = cpos;
@@ -148,11 +148,11 @@ cudaError_t launch_pair_histogram(const int32_t* idx, int P, int E, int32_t* chu
 }
 
 cudaError_t launch_expert_scan(int NC, int E, int32_t* chunk_hist, int32_t* counts, int32_t* offsets,
-                               int32_t* touched, int32_t* group_base, int32_t* tile_base, int32_t* meta,
-                               cudaStream_t s) {
+                               int32_t* touched, int32_t* group_base, int32_t* tile_base, int chunk,
+                               int32_t* meta, cudaStream_t s) {
   const int threads = ((E + 31) / 32) * 32;
   expert_scan_kernel<<<1, threads, 0, s>>>(NC, E, chunk_hist, counts, offsets, touched, group_base, tile_base,
-                                           meta);
+                                           chunk, meta);
   return cudaGetLastError();
 }
 

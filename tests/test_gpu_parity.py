@@ -20,7 +20,8 @@ PATHS = {"auto": moe.MOE_PATH_AUTO, "gemv": moe.MOE_PATH_GEMV, "gemm": moe.MOE_P
 SMALL = {
     "tiny-fp32": (1, {}),
     "kimi-bf16-small": (2, dict(T=37, H=256, E=32, I=256)),
-    "kimi-bf16-ragged": (2, dict(T=45, H=256, E=32, I=192)),      # I not a multiple of 128: GEMV only
+    "kimi-bf16-ragged": (2, dict(T=45, H=256, E=32, I=192)),      # I a multiple of 64, not of 128
+    "kimi-bf16-odd-H": (2, dict(T=29, H=320, E=16, I=128)),       # H not a multiple of 128: GEMV only
     "kimi-int8-small": (3, dict(T=203, H=384, E=24, I=256)),
     "qwen3-int4-small": (4, dict(T=150, H=256, E=16, I=128)),
     "skew-masked-int8-small": (5, dict(T=301, H=256, E=40, I=128, n_active=23, bias=("skew", 0.15))),
@@ -39,7 +40,7 @@ def _clear_flags():
 def test_small_workloads(name, path):
     cid, over = SMALL[name]
     prob = synth.make_problem(cid, **over)
-    if path == "gemm" and (prob.wfmt == "f32" or prob.H % 128 or prob.I % 128):
+    if path == "gemm" and (prob.wfmt == "f32" or prob.H % 128 or prob.I % 64):
         with pytest.raises(moe.MoeError) as ei:
             run(prob, PATHS[path])
         assert ei.value.status == moe.MOE_ERR_UNSUPPORTED
