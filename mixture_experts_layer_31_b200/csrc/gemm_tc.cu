@@ -8,10 +8,10 @@
 // M = 128 and N = the chunk's token count rounded up to 16 (<= 256), so a
 // ragged expert pays at most 15 padded columns.
 //
-//   gate/up: the 128 A rows are 64 rows of W_gate and the same 64 rows of
-//            W_up, so one accumulator holds both projections of 64 outputs:
-//            h[pos, i] = SiLU(s_g D[i, pos]) * (s_u D[64 + i, pos])  (bf16 out)
-//   down:    A = 128 rows of W_down;  Yp[pair, r] = w_pair * s_d * D[r, pos] (fp32)
+//   gate/up: M tile 0 = 128 rows of W_gate, M tile 1 = the same rows of W_up,
+//            both against one token tile, so TMEM lane i holds both projections
+//            of output row i:  h[pos, i] = SiLU(s_g D0[i, pos]) * (s_u D1[i, pos])
+//   down:    1 or 2 M tiles of 128 W_down rows;  Yp[pair, r] = w_pair * s_d * D[r, pos]
 // Storage: bf16 weights go straight from TMA into the 128-byte-swizzled
 // K-major layout the tensor core reads; int8 rows (one scale per row and
 // expert -- Kimi-Linear LiteRT-LM details, quantization bullet) are widened
@@ -21,10 +21,11 @@
 // Roles in a persistent CTA (one per SM), all walking one list of units:
 //   warp 0 lane 0   TMA producer (weight or raw quantised tiles, token boxes)
 //   warp 1          TMEM allocator; lane 0 issues tcgen05.mma, commits stages
-//   warps 4..7      epilogue: tcgen05.ld -> activation / scales -> global
-//   warps 8..15     dequantisation (int8 / int4 only)
-// TMEM holds two accumulators of `chunk` columns, so the epilogue of one unit
-// overlaps the MMAs of the next.  Every wait is bounded (MOE_FLAG_TIMEOUT).
+//   warps 4..11     epilogue (two 4-warp groups): tcgen05.ld -> activation / scales -> global
+//   warps 12..19    dequantisation (int8 / int4 only)
+// TMEM holds two accumulator buffers when they fit (chunks up to 128 tokens),
+// so the epilogue of one unit overlaps the MMAs of the next.  Every wait is
+// bounded (MOE_FLAG_TIMEOUT).
 // No cluster, no multicast.
 #include <cuda.h>
 
@@ -40,8 +41,6 @@ constexpr int kTileBytes = kBM * kBK * 2;  // A tile, 16 KB
 constexpr int kBoxRows = 32;               // token rows per TMA box
 constexpr int kMaxStages = 8;
 constexpr int kAStages = 2;                // quantised: bf16 A tiles between dequant and MMA
-constexpr int kXchgCols = 16;              // gate/up epilogue exchange: columns per step
-constexpr int kXchgBytes = 2 * kXchgCols * 64 * 4;  // double-buffered [16 cols][64 rows] fp32
 constexpr int kBarrierBytes = 1024;
 constexpr int kSmemLimit = 232448;         // 227 KB opt-in
 
@@ -138,18 +137,16 @@ __device__ __forceinline__ uint4 widen8(const uint8_t* raw_chunk, float scale) {
 template <int MODE, int WF, int MT>
 struct Traits {
   static constexpr bool kQuant = WF != MOE_W_BF16;
-  static constexpr int kTileRows = MODE == 0 ? 64 : 128;  // output rows per M tile
-  static constexpr int kRows = kTileRows * MT;            // output rows per unit
+  // gate/up: MT = 2 (gate tile, up tile) over 128 output rows; down: MT tiles of 128 rows
+  static constexpr int kRows = MODE == 0 ? kBM : kBM * MT;  // output rows per unit
   static constexpr int kRawTile = WF == MOE_W_INT8_ROW ? kBM * kBK : (WF == MOE_W_INT4_B32 ? kBM * kBK / 2 : 0);
   static constexpr int kRawPitch = WF == MOE_W_INT8_ROW ? kBK : kBK / 2;  // bytes per raw row
-  static constexpr int kEpiWarps = 4 * MT;                // one 4-warp group per M tile
+  static constexpr int kEpiWarps = 8;                     // two 4-warp groups
   static constexpr int kDequantWarps = kQuant ? 8 : 0;
   static constexpr int kDequant0 = 4 + kEpiWarps;         // first dequant warp
   static constexpr int kThreads = 32 * (4 + kEpiWarps + kDequantWarps);
-  // per group: gate/up exchange of up values between TMEM quadrants (8 KB);
-  // down: the unit's pair ids and routing weights (2 KB)
-  static constexpr int kGroupXchg = MODE == 0 ? kXchgBytes : 2 * 256 * 4;
-  static constexpr int kXchg = (MT * kGroupXchg + 1023) / 1024 * 1024;
+  static constexpr int kGroupXchg = MODE == 0 ? 0 : 2 * 256 * 4;  // down: pair ids + weights per group
+  static constexpr int kXchg = (2 * kGroupXchg + 1023) / 1024 * 1024;
 };
 
 template <int MODE, int WF, int MT>
@@ -203,7 +200,7 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int ntouched = a.meta[0];
-  const int nib = a.R / Tr::kRows;
+  const int nib = (a.R + Tr::kRows - 1) / Tr::kRows;  // gate/up: the last block may be half (I % 128 == 64)
   const int total = ntouched > 0 ? a.meta[3] * nib : 0;
   const int nk = a.K / kBK;
 
@@ -228,14 +225,10 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
 #pragma unroll
           for (int mt = 0; mt < MT; ++mt) {
             uint8_t* adst = Tr::kQuant ? st + a.raw_off + mt * Tr::kRawTile : st + mt * kTileBytes;
-            const int wrow = wrow0 + mt * Tr::kTileRows;
-            if (MODE == 0) {
-              const int half = Tr::kQuant ? 64 * Tr::kRawPitch : kTileBytes / 2;
-              tma_load_2d(adst, &tm_w0, wcol, wrow, &full[s]);         // 64 gate rows
-              tma_load_2d(adst + half, &tm_w1, wcol, wrow, &full[s]);  // the same 64 up rows
-            } else {
-              tma_load_2d(adst, &tm_w0, wcol, wrow, &full[s]);         // 128 down rows
-            }
+            if (MODE == 0)  // tile 0: 128 gate rows, tile 1: the same 128 up rows
+              tma_load_2d(adst, mt ? &tm_w1 : &tm_w0, wcol, wrow0, &full[s]);
+            else            // 128 down rows per tile
+              tma_load_2d(adst, &tm_w0, wcol, wrow0 + mt * kBM, &full[s]);
           }
           for (int j = 0; j < nbox; ++j)
             tma_load_2d(st + a.b_off + j * kBoxRows * kBK * 2, &tm_b, kb * kBK, brow + kBoxRows * j, &full[s]);
@@ -287,46 +280,49 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
     }
   } else if (w >= 4 && w < 4 + Tr::kEpiWarps) {
     // ------------------------------------------------------------------ epilogue
-    const int grp = (w - 4) >> 2;  // M tile drained by this 4-warp group
-    const int q = w & 3;           // TMEM lanes 32q .. 32q+31
+    // Each thread owns one TMEM lane = one output row.  Gate/up and single-tile
+    // down: the two groups split the unit's 16-column chunks (even / odd);
+    // two-tile down: group g drains tile g.
+    const int grp = (w - 4) >> 2;
+    const int q = w & 3;  // TMEM lanes 32q .. 32q+31
+    const bool split_cols = MODE == 0 || MT == 1;
     const int bar_x = 1 + 2 * grp, bar_v = 2 + 2 * grp;
     float* gx = xchg + grp * (Tr::kGroupXchg / 4);
     bool dead = false;
-    uint32_t local = 0, xc = 0;
+    uint32_t local = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x, ++local) {
       const Unit t = decode_unit(a, u, nib, ntouched);
       const uint32_t buf = local % nbuf;
       if (lane == 0) wait_or_die(&acc_full[buf], (local / nbuf) & 1u, dead, a.flags);
-      // the group's four warps agree on the verdict (their loops hold named barriers)
-      dead = named_bar_or(bar_v, 128, dead);
+      if (MODE == 0) {
+        dead = __shfl_sync(0xFFFFFFFFu, dead ? 1 : 0, 0) != 0;
+        __syncwarp();
+      } else {
+        dead = named_bar_or(bar_v, 128, dead);  // the group stages shared pair ids below
+      }
       tc_fence_after();
-      const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * buf_cols + grp * a.acc_stride;
+      const int tile = split_cols ? 0 : grp;
+      const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * buf_cols + tile * a.acc_stride;
       const int pos0 = t.base + t.c * a.chunk;
+      const int c_first = split_cols ? grp * 16 : 0, c_step = split_cols ? 32 : 16;
       if (!dead) {
         if (MODE == 0) {
-          // lanes 0..63 hold gate rows, 64..127 the matching up rows: up warps hand
-          // their values to the gate warps through a double-buffered exchange
-          const int r64 = (q & 1) * 32 + lane;
-          const int row = t.ib * Tr::kRows + grp * 64 + r64;
-          const size_t grow = (size_t)t.e * a.R + row;
+          const int row = t.ib * kBM + q * 32 + lane;
+          const bool live = row < a.R;
+          const size_t grow = (size_t)t.e * a.R + (live ? row : 0);
           const float sg = WF == MOE_W_INT8_ROW ? a.s0[grow] : 1.f;
           const float su = WF == MOE_W_INT8_ROW ? a.s1[grow] : 1.f;
           uint16_t* hout = static_cast<uint16_t*>(a.out);
-          for (int n0 = 0; n0 < t.n_tok; n0 += kXchgCols, ++xc) {
-            float* xb = gx + (xc & 1u) * (kXchgCols * 64);
-            uint32_t v[16];
-            tmem_ld16(tacc + n0, v);
+          for (int n0 = c_first; n0 < t.n_tok; n0 += c_step) {
+            uint32_t g[16], v[16];
+            tmem_ld16(tacc + n0, g);
+            tmem_ld16(tacc + a.acc_stride + n0, v);
             tmem_ld_wait();
-            if (q >= 2) {
-#pragma unroll
-              for (int j = 0; j < 16; ++j) xb[j * 64 + r64] = __uint_as_float(v[j]);
-            }
-            named_bar_sync(bar_x, 128);
-            if (q < 2) {
+            if (live) {
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
                 if (n0 + j < t.n_tok) {
-                  const float hv = silu_mul_fast(__uint_as_float(v[j]) * sg, xb[j * 64 + r64] * su);
+                  const float hv = silu_mul_fast(__uint_as_float(g[j]) * sg, __uint_as_float(v[j]) * su);
                   hout[(size_t)(pos0 + n0 + j) * a.R + row] = f32_to_bf16(hv);
                 }
               }
@@ -343,10 +339,10 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
             s_w[n] = a.topk_w[pair];
           }
           named_bar_sync(bar_x, 128);
-          const int row = t.ib * Tr::kRows + grp * 128 + et;
+          const int row = t.ib * Tr::kRows + tile * kBM + et;
           const float sd = WF == MOE_W_INT8_ROW ? a.s0[(size_t)t.e * a.R + row] : 1.f;
           float* yp = static_cast<float*>(a.out);
-          for (int n0 = 0; n0 < t.n_tok; n0 += 16) {
+          for (int n0 = c_first; n0 < t.n_tok; n0 += c_step) {
             uint32_t v[16];
             tmem_ld16(tacc + n0, v);
             tmem_ld_wait();
@@ -382,8 +378,9 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
       for (int j = 0; j < kPer; ++j) {
         const int r = r0 + kRowStep * j;  // row within the unit's MT*128 A rows
         const int mt = r >> 7, rr = r & 127;
-        const float* S = (MODE == 0 && rr >= 64) ? a.s1 : a.s0;
-        const int wr = t.ib * Tr::kRows + mt * Tr::kTileRows + (MODE == 0 ? (rr & 63) : rr);
+        const float* S = (MODE == 0 && mt == 1) ? a.s1 : a.s0;
+        int wr = MODE == 0 ? t.ib * kBM + rr : t.ib * Tr::kRows + mt * kBM + rr;
+        if (wr >= a.R) wr = a.R - 1;  // rows past a half block are computed but never stored
         srow[j] = S + ((size_t)t.e * a.R + wr) * (a.K / 32) + (c8 >> 2);
         sc_next[j] = WF == MOE_W_INT4_B32 ? __ldg(srow[j]) : 1.f;
       }
@@ -496,14 +493,14 @@ cudaError_t launch_gemm(const CUtensorMap& m0, const CUtensorMap& m1, const CUte
   return cudaGetLastError();
 }
 
-// two M tiles per unit (B reused across 256 weight rows) once chunks are large
-// enough for the tensor core to be the bottleneck; one tile for small batches,
-// where finer units balance the weight stream across SMs
+// gate/up always carries two M tiles (gate, up); down carries two tiles of W_down
+// rows once chunks are large enough for the tensor core to bind (the token tile
+// then feeds 256 weight rows), one for small batches, where finer units balance
+// the weight stream across SMs
 template <int MODE>
 cudaError_t launch_by_format(int wfmt, const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb,
                              const GemmArgs& a, int num_sms, cudaStream_t s) {
-  const int tile_rows = MODE == 0 ? 64 : 128;
-  const bool two = a.chunk >= 128 && a.R % (2 * tile_rows) == 0;
+  const bool two = MODE == 0 || (a.chunk >= 128 && a.R % (2 * kBM) == 0);
   switch (wfmt) {
     case MOE_W_BF16:
       return two ? launch_gemm<MODE, MOE_W_BF16, 2>(m0, m1, mb, a, num_sms, s)
@@ -544,7 +541,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
 
 }  // namespace
 
-// gate/up tiles 64 output rows (K = H); down tiles 128 rows of H (K = I)
+// gate/up tiles 128 output rows of I (a multiple of 64; a half block is computed
+// and not stored); down tiles 128 rows of H (K = I)
 bool gemm_tc_supported(const moe_desc& d) {
   return d.xfmt == MOE_X_BF16 && d.wfmt != MOE_W_F32 && d.H % 128 == 0 && d.I % 64 == 0 && encode_fn() != nullptr;
 }
@@ -563,8 +561,8 @@ cudaError_t launch_gather_rows(const moe_desc& d, const void* x, const Workspace
 cudaError_t launch_gemm_gateup(const moe_desc& d, const Workspace& ws, int P, int chunk, int num_sms,
                                uint32_t* flags, cudaStream_t s) {
   CUtensorMap mg, mu, mb;
-  cudaError_t e = weight_map(&mg, d.W_gate, d.wfmt, d.E, d.I, d.H, 64);
-  if (e == cudaSuccess) e = weight_map(&mu, d.W_up, d.wfmt, d.E, d.I, d.H, 64);
+  cudaError_t e = weight_map(&mg, d.W_gate, d.wfmt, d.E, d.I, d.H, kBM);
+  if (e == cudaSuccess) e = weight_map(&mu, d.W_up, d.wfmt, d.E, d.I, d.H, kBM);
   if (e == cudaSuccess)
     e = make_map(&mb, ws.xs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.H, (uint64_t)P, kBK, kBoxRows,
                  CU_TENSOR_MAP_SWIZZLE_128B);
