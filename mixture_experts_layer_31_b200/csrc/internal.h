@@ -20,10 +20,14 @@ constexpr int kGemvGroup = 4;
 // kMaxTileN (the N of one MMA tile).  A batch of T tokens routes at most T
 // of them to one expert, so small batches use smaller chunks (and smaller
 // pipeline stages): chunk = min(kMaxTileN, T rounded up to 16).
+// Chunks above 128 tokens leave room for only one TMEM accumulator buffer (no
+// epilogue overlap); batches averaging <= 96 tokens per expert use 128.
 constexpr int kMaxTileN = 256;
-inline int chunk_tokens(int T) {
-  const int t = ((T > 0 ? T : 1) + 15) / 16 * 16;
-  return t < kMaxTileN ? t : kMaxTileN;
+inline int chunk_tokens(int T, int k, int E) {
+  int t = ((T > 0 ? T : 1) + 15) / 16 * 16;
+  if (t > kMaxTileN) t = kMaxTileN;
+  if (t > 128 && (long long)T * k <= 96LL * E) t = 128;
+  return t;
 }
 
 // Split of the router's reduction over H into S partial sums (summed in a
@@ -63,6 +67,10 @@ cudaError_t launch_router_logits(const moe_desc& d, const void* x, int T, float*
                                  cudaStream_t s);
 cudaError_t launch_router_topk(const moe_desc& d, const float* partial, int S, int T, int32_t* idx,
                                float* w, uint32_t* flags, cudaStream_t s);
+bool small_sort_ok(int P, int E);
+cudaError_t launch_small_sort(const int32_t* idx, int P, int E, int chunk, int32_t* counts, int32_t* offsets,
+                              int32_t* touched, int32_t* group_base, int32_t* tile_base, int32_t* meta,
+                              int32_t* sorted_pair, uint32_t* flags, cudaStream_t s);
 cudaError_t launch_pair_histogram(const int32_t* idx, int P, int E, int32_t* chunk_hist,
                                   uint32_t* flags, cudaStream_t s);
 cudaError_t launch_expert_scan(int NC, int E, int32_t* chunk_hist, int32_t* counts, int32_t* offsets,

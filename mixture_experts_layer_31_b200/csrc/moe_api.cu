@@ -295,14 +295,20 @@ extern "C" moe_status moe_forward(const moe_desc* d, const void* x, int32_t T, c
   const Workspace ws = carve_workspace(*d, T, workspace);
   const int P = T * d->k;
   const int NC = (P + kPairChunk - 1) / kPairChunk;
-  MOE_LAUNCH("pair_histogram", stream, launch_pair_histogram(topk_idx, P, d->E, ws.chunk_hist, dev->flags, stream));
-  MOE_LAUNCH("expert_scan", stream,
-             launch_expert_scan(NC, d->E, ws.chunk_hist, ws.counts, ws.offsets, ws.touched, ws.group_base,
-                                ws.tile_base, chunk_tokens(T), ws.meta, stream));
-  MOE_LAUNCH("pair_scatter", stream, launch_pair_scatter(topk_idx, P, d->E, ws.chunk_hist, ws.sorted_pair, stream));
+  if (small_sort_ok(P, d->E)) {
+    MOE_LAUNCH("small_sort", stream,
+               launch_small_sort(topk_idx, P, d->E, chunk_tokens(T, d->k, d->E), ws.counts, ws.offsets, ws.touched,
+                                 ws.group_base, ws.tile_base, ws.meta, ws.sorted_pair, dev->flags, stream));
+  } else {
+    MOE_LAUNCH("pair_histogram", stream, launch_pair_histogram(topk_idx, P, d->E, ws.chunk_hist, dev->flags, stream));
+    MOE_LAUNCH("expert_scan", stream,
+               launch_expert_scan(NC, d->E, ws.chunk_hist, ws.counts, ws.offsets, ws.touched, ws.group_base,
+                                  ws.tile_base, chunk_tokens(T, d->k, d->E), ws.meta, stream));
+    MOE_LAUNCH("pair_scatter", stream, launch_pair_scatter(topk_idx, P, d->E, ws.chunk_hist, ws.sorted_pair, stream));
+  }
   if (path == MOE_PATH_GEMM) {
     MOE_LAUNCH("gather_rows", stream, launch_gather_rows(*d, x, ws, P, dev->num_sms, stream));
-    const int chunk = chunk_tokens(T);
+    const int chunk = chunk_tokens(T, d->k, d->E);
     MOE_LAUNCH("gemm_gateup", stream, launch_gemm_gateup(*d, ws, P, chunk, dev->num_sms, dev->flags, stream));
     MOE_LAUNCH("gemm_down", stream, launch_gemm_down(*d, topk_w, ws, P, chunk, dev->num_sms, dev->flags, stream));
   } else {

@@ -51,10 +51,10 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const void* __restri
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 
-  for (int k0 = kb; k0 < ke; k0 += kBK) {
-    float xv[8], wv[8];
+  // global -> registers for the K tile at k0 (zero outside the matrix)
+  auto fetch = [&](int k0, float (&xv)[8], float (&wv)[8]) {
     const int t = t0 + lr;
-    if (t < T) {
+    if (t < T && k0 < ke) {
       if (XBF16) {
         const uint4 v = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + (size_t)t * H + k0 + lq);
         const uint32_t u[4] = {v.x, v.y, v.z, v.w};
@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const void* __restri
       for (int j = 0; j < 8; ++j) xv[j] = 0.f;
     }
     const int e = e0 + lr;
-    if (e < E) {
+    if (e < E && k0 < ke) {
       const float4* p = reinterpret_cast<const float4*>(Wr + (size_t)e * H + k0 + lq);
       const float4 a = p[0], b = p[1];
       wv[0] = a.x; wv[1] = a.y; wv[2] = a.z; wv[3] = a.w;
@@ -83,12 +83,17 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const void* __restri
 #pragma unroll
       for (int j = 0; j < 8; ++j) wv[j] = 0.f;
     }
+  };
+  float xv[8], wv[8];
+  fetch(kb, xv, wv);
+  for (int k0 = kb; k0 < ke; k0 += kBK) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       xs[lq + j][lr] = xv[j];
       wsm[lq + j][lr] = wv[j];
     }
     __syncthreads();
+    fetch(k0 + kBK, xv, wv);  // next tile's loads overlap this tile's FMAs
 #pragma unroll
     for (int kk = 0; kk < kBK; ++kk) {
       const float4 a = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
@@ -119,8 +124,8 @@ __device__ __forceinline__ bool better(float ka, int ea, float kb, int eb) {
   return ka > kb || (ka == kb && ea < eb);
 }
 
-template <int PER_LANE>
-__global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ partial, int S, int T,
+template <int PER_LANE, int S>
+__global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ partial, int T,
                                                           int E, int k, int router,
                                                           const float* __restrict__ bias,
                                                           const uint8_t* __restrict__ mask, float scale,
@@ -132,6 +137,13 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
   float logit[PER_LANE], key[PER_LANE];
   uint32_t avail = 0;
   bool bad = false;
+  // issue every partial load before summing (split sums in a fixed order)
+  float part[PER_LANE][S];
+#pragma unroll
+  for (int j = 0; j < PER_LANE; ++j)
+#pragma unroll
+    for (int s = 0; s < S; ++s)
+      part[j][s] = (lane + 32 * j < E) ? partial[((size_t)s * T + t) * E + lane + 32 * j] : 0.f;
 #pragma unroll
   for (int j = 0; j < PER_LANE; ++j) {
     const int e = lane + 32 * j;
@@ -139,7 +151,8 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
     key[j] = -INFINITY;
     if (e < E) {
       float l = 0.f;
-      for (int s = 0; s < S; ++s) l += partial[((size_t)s * T + t) * E + e];
+#pragma unroll
+      for (int s = 0; s < S; ++s) l += part[j][s];
       logit[j] = l;
       const bool active = (mask == nullptr) || (mask[e] != 0);
       if (!isfinite(l)) {
@@ -226,12 +239,25 @@ cudaError_t launch_router_topk(const moe_desc& d, const float* partial, int S, i
                                float* w, uint32_t* flags, cudaStream_t s) {
   const int warps = 8;
   dim3 grid((T + warps - 1) / warps);
-  if (d.E <= 256)
-    router_topk_kernel<8><<<grid, warps * 32, 0, s>>>(partial, S, T, d.E, d.k, d.router, d.b, d.expert_mask,
-                                                      d.scale, idx, w, flags);
-  else
-    router_topk_kernel<32><<<grid, warps * 32, 0, s>>>(partial, S, T, d.E, d.k, d.router, d.b,
-                                                       d.expert_mask, d.scale, idx, w, flags);
+#define MOE_TOPK(PL, SS)                                                                                 \
+  router_topk_kernel<PL, SS><<<grid, warps * 32, 0, s>>>(partial, T, d.E, d.k, d.router, d.b, d.expert_mask, \
+                                                         d.scale, idx, w, flags)
+  if (d.E <= 256) {
+    switch (S) {
+      case 1: MOE_TOPK(8, 1); break;
+      case 2: MOE_TOPK(8, 2); break;
+      case 4: MOE_TOPK(8, 4); break;
+      default: MOE_TOPK(8, 8); break;
+    }
+  } else {
+    switch (S) {
+      case 1: MOE_TOPK(32, 1); break;
+      case 2: MOE_TOPK(32, 2); break;
+      case 4: MOE_TOPK(32, 4); break;
+      default: MOE_TOPK(32, 8); break;
+    }
+  }
+#undef MOE_TOPK
   return cudaGetLastError();
 }
 

@@ -22,6 +22,7 @@ SMALL = {
     "kimi-bf16-small": (2, dict(T=37, H=256, E=32, I=256)),
     "kimi-bf16-ragged": (2, dict(T=45, H=256, E=32, I=192)),      # I a multiple of 64, not of 128
     "kimi-bf16-odd-H": (2, dict(T=29, H=320, E=16, I=128)),       # H not a multiple of 128: GEMV only
+    "kimi-bf16-wide-E": (2, dict(T=40, H=256, E=320, I=128)),     # E > 256: wide top-k, chunked sort
     "kimi-int8-small": (3, dict(T=203, H=384, E=24, I=256)),
     "qwen3-int4-small": (4, dict(T=150, H=256, E=16, I=128)),
     "skew-masked-int8-small": (5, dict(T=301, H=256, E=40, I=128, n_active=23, bias=("skew", 0.15))),
@@ -75,6 +76,15 @@ def test_full_workloads_sampled(cid, n_sample):
     judge(prob, y, idx, w, tokens=toks)
     if prob.mask is not None:
         assert prob.mask[idx.cpu().numpy()].all()
+
+
+@pytest.mark.parametrize("T", [1000, 1100])
+def test_sort_paths_agree_with_oracle(T):
+    """P = 8000 takes the single-CTA sort, P = 8800 the chunked one; both must
+    give the oracle's result."""
+    prob = synth.make_problem(4, T=T, H=256, E=64, I=128)
+    _, _, y, idx, w = run(prob)
+    judge(prob, y, idx, w, tokens=np.arange(0, T, 7))
 
 
 def test_deterministic_repeat():
@@ -183,5 +193,8 @@ def test_stage_timing_reports_every_kernel():
         times = moe.moe_stage_times()
     finally:
         moe.moe_stage_timing(False)
-    for name in ("router_logits", "router_topk", "pair_histogram", "expert_scan", "pair_scatter", "combine"):
+    for name in ("router_logits", "router_topk", "combine"):
+        assert name in times and times[name][0] == 1 and times[name][1] > 0
+    sort = ("small_sort",) if "small_sort" in times else ("pair_histogram", "expert_scan", "pair_scatter")
+    for name in sort:
         assert name in times and times[name][0] == 1 and times[name][1] > 0
