@@ -65,6 +65,10 @@ struct GemmArgs {
   int acc_stride;       // TMEM columns per M tile accumulator (power of two >= chunk)
   int nbuf;             // accumulator buffers (2: epilogue overlaps the next unit's MMAs)
   int tmem_cols;        // TMEM columns allocated
+  // router logits (MODE 2): dense [T, E] = x [T, H] . W3 [E, 3H]^T over S splits of the K steps
+  int T;
+  int S;
+  int Hx;               // columns of x (the K coordinate of x is taken modulo Hx)
 };
 
 __device__ __forceinline__ void wait_or_die(uint64_t* bar, uint32_t parity, bool& dead, uint32_t* flags) {
@@ -77,17 +81,33 @@ __device__ __forceinline__ void wait_or_die(uint64_t* bar, uint32_t parity, bool
 
 struct Unit {
   int e, base, ib, c, n_tok, n_mma;
+  int k0, nk;  // K steps [k0, k0 + nk)
 };
 
-// unit u -> (expert, output-row block, token chunk); chunks fastest
+// units of the expert GEMMs (MODE 0/1): (expert, output-row block, token chunk),
+// chunks fastest; of the router GEMM (MODE 2): (token chunk, expert block, K split)
+template <int MODE>
 __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u, int nib, int ntouched) {
+  Unit t;
+  const int nk_all = a.K / kBK;
+  if (MODE == 2) {
+    const int s = u % a.S, r = u / a.S;
+    t.ib = r % nib;
+    t.c = s;
+    t.e = 0;
+    t.base = (r / nib) * a.chunk;
+    t.n_tok = min(a.chunk, a.T - t.base);
+    t.n_mma = (t.n_tok + 15) & ~15;
+    t.k0 = s * nk_all / a.S;
+    t.nk = (s + 1) * nk_all / a.S - t.k0;
+    return t;
+  }
   int lo = 0, hi = ntouched - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (a.tile_base[mid] * nib <= u) lo = mid;
     else hi = mid - 1;
   }
-  Unit t;
   t.e = a.touched[lo];
   t.base = a.offsets[t.e];
   const int m = a.offsets[t.e + 1] - t.base;
@@ -97,6 +117,8 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u, int nib, i
   t.c = r - t.ib * nc;
   t.n_tok = min(a.chunk, m - t.c * a.chunk);
   t.n_mma = (t.n_tok + 15) & ~15;
+  t.k0 = 0;
+  t.nk = nk_all;
   return t;
 }
 
@@ -199,10 +221,10 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int ntouched = a.meta[0];
+  const int ntouched = MODE == 2 ? 0 : a.meta[0];
   const int nib = (a.R + Tr::kRows - 1) / Tr::kRows;  // gate/up: the last block may be half (I % 128 == 64)
-  const int total = ntouched > 0 ? a.meta[3] * nib : 0;
-  const int nk = a.K / kBK;
+  const int total = MODE == 2 ? nib * ((a.T + a.chunk - 1) / a.chunk) * a.S
+                              : (ntouched > 0 ? a.meta[3] * nib : 0);
 
   if (w == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -211,11 +233,11 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
       uint32_t it = 0;
       const uint32_t abytes = MT * (Tr::kQuant ? Tr::kRawTile : kTileBytes);
       for (int u = blockIdx.x; u < total; u += gridDim.x) {
-        const Unit t = decode_unit(a, u, nib, ntouched);
+        const Unit t = decode_unit<MODE>(a, u, nib, ntouched);
         const int nbox = (t.n_tok + kBoxRows - 1) / kBoxRows;
-        const int brow = t.base + t.c * a.chunk;
+        const int brow = MODE == 2 ? t.base : t.base + t.c * a.chunk;
         const int wrow0 = t.e * a.R + t.ib * Tr::kRows;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        for (int kb = t.k0; kb < t.k0 + t.nk; ++kb, ++it) {
           const int s = it % NS;
           wait_or_die(&empty[s], ((it / NS) & 1u) ^ 1u, dead, a.flags);
           if (dead) continue;
@@ -230,8 +252,9 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
             else            // 128 down rows per tile
               tma_load_2d(adst, &tm_w0, wcol, wrow0 + mt * kBM, &full[s]);
           }
+          const int bcol = MODE == 2 ? (kb * kBK) % a.Hx : kb * kBK;
           for (int j = 0; j < nbox; ++j)
-            tma_load_2d(st + a.b_off + j * kBoxRows * kBK * 2, &tm_b, kb * kBK, brow + kBoxRows * j, &full[s]);
+            tma_load_2d(st + a.b_off + j * kBoxRows * kBK * 2, &tm_b, bcol, brow + kBoxRows * j, &full[s]);
         }
       }
       const uint32_t first = it > (uint32_t)NS ? it - NS : 0u;
@@ -245,13 +268,13 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
       const uint32_t stage0 = smem_u32(stages);
       const uint32_t a_ring0 = smem_u32(a_ring);
       for (int u = blockIdx.x; u < total; u += gridDim.x, ++local) {
-        const Unit t = decode_unit(a, u, nib, ntouched);
+        const Unit t = decode_unit<MODE>(a, u, nib, ntouched);
         const uint32_t buf = local % nbuf;
         wait_or_die(&acc_empty[buf], ((local / nbuf) & 1u) ^ 1u, dead, a.flags);
         tc_fence_after();
         const uint32_t idesc = umma_idesc_bf16(kBM, t.n_mma);
         const uint32_t d = tmem_base + buf * buf_cols;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        for (int kb = 0; kb < t.nk; ++kb, ++it) {
           const int s = it % NS;
           const int ja = it % kAStages;
           if (Tr::kQuant) wait_or_die(&ready[ja], (it / kAStages) & 1u, dead, a.flags);
@@ -285,16 +308,16 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
     // two-tile down: group g drains tile g.
     const int grp = (w - 4) >> 2;
     const int q = w & 3;  // TMEM lanes 32q .. 32q+31
-    const bool split_cols = MODE == 0 || MT == 1;
+    const bool split_cols = MODE != 1 || MT == 1;
     const int bar_x = 1 + 2 * grp, bar_v = 2 + 2 * grp;
     float* gx = xchg + grp * (Tr::kGroupXchg / 4);
     bool dead = false;
     uint32_t local = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x, ++local) {
-      const Unit t = decode_unit(a, u, nib, ntouched);
+      const Unit t = decode_unit<MODE>(a, u, nib, ntouched);
       const uint32_t buf = local % nbuf;
       if (lane == 0) wait_or_die(&acc_full[buf], (local / nbuf) & 1u, dead, a.flags);
-      if (MODE == 0) {
+      if (MODE != 1) {
         dead = __shfl_sync(0xFFFFFFFFu, dead ? 1 : 0, 0) != 0;
         __syncwarp();
       } else {
@@ -326,6 +349,20 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
                   hout[(size_t)(pos0 + n0 + j) * a.R + row] = f32_to_bf16(hv);
                 }
               }
+            }
+          }
+        } else if (MODE == 2) {
+          // router logits: partial[s][t][e] (fp32), tokens along columns
+          const int e = t.ib * kBM + q * 32 + lane;
+          float* part = static_cast<float*>(a.out) + (size_t)t.c * a.T * a.R;
+          for (int n0 = c_first; n0 < t.n_tok; n0 += c_step) {
+            uint32_t v[16];
+            tmem_ld16(tacc + n0, v);
+            tmem_ld_wait();
+            if (e < a.R) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                if (n0 + j < t.n_tok) part[(size_t)(t.base + n0 + j) * a.R + e] = __uint_as_float(v[j]);
             }
           }
         } else {
@@ -370,7 +407,7 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
     bool dead = false;
     uint32_t it = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
-      const Unit t = decode_unit(a, u, nib, ntouched);
+      const Unit t = decode_unit<MODE>(a, u, nib, ntouched);
       // int4: block scales of this thread's rows, one K step ahead
       const float* srow[kPer];
       float sc_next[kPer];
@@ -384,12 +421,12 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
         srow[j] = S + ((size_t)t.e * a.R + wr) * (a.K / 32) + (c8 >> 2);
         sc_next[j] = WF == MOE_W_INT4_B32 ? __ldg(srow[j]) : 1.f;
       }
-      for (int kb = 0; kb < nk; ++kb, ++it) {
+      for (int kb = 0; kb < t.nk; ++kb, ++it) {
         float sc[kPer];
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
           sc[j] = sc_next[j];
-          if (WF == MOE_W_INT4_B32 && kb + 1 < nk) sc_next[j] = __ldg(srow[j] + (kb + 1) * 2);
+          if (WF == MOE_W_INT4_B32 && kb + 1 < t.nk) sc_next[j] = __ldg(srow[j] + (kb + 1) * 2);
         }
         const int s = it % NS;
         const int ja = it % kAStages;
@@ -539,7 +576,72 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
   }
 }
 
+// W3[e] = [hi | mid | lo] with hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid):
+// each difference is exact in fp32 and the three parts reproduce w to ~2^-27
+// relative, so bf16 x against W3 over 3H columns gives fp32-accurate logits
+__global__ void __launch_bounds__(256) split3_kernel(const float* __restrict__ Wr, int E, int H,
+                                                     uint16_t* __restrict__ W3) {
+  const size_t n = (size_t)E * H;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const size_t e = i / H, h = i - e * H;
+    const float w = Wr[i];
+    const uint16_t hi = f32_to_bf16(w);
+    const float r1 = w - bf16_to_f32(hi);
+    const uint16_t mid = f32_to_bf16(r1);
+    const float r2 = r1 - bf16_to_f32(mid);
+    uint16_t* row = W3 + e * 3 * H;
+    row[h] = hi;
+    row[H + h] = mid;
+    row[2 * H + h] = f32_to_bf16(r2);
+  }
+}
+
 }  // namespace
+
+int router_tc_chunk(int T) {
+  const int t = ((T > 0 ? T : 1) + 15) / 16 * 16;
+  return t < kMaxTileN ? t : kMaxTileN;
+}
+
+// K splits of the tensor-core router: a function of T only, so a masked layer and
+// its sliced twin sum identical partials in the same order
+int router_tc_splits(int T) {
+  const int chunks = (T + router_tc_chunk(T) - 1) / router_tc_chunk(T);
+  int S = 1;
+  while (S < 8 && chunks * S * 2 <= 74) S *= 2;
+  return S;
+}
+
+bool router_tc_supported(const moe_desc& d) { return d.xfmt == MOE_X_BF16 && encode_fn() != nullptr; }
+
+cudaError_t launch_router_split3(const moe_desc& d, void* W3, int num_sms, cudaStream_t s) {
+  const size_t n = (size_t)d.E * d.H;
+  int blocks = (int)((n + 255) / 256);
+  if (blocks > num_sms * 4) blocks = num_sms * 4;
+  split3_kernel<<<blocks, 256, 0, s>>>(d.W_r, d.E, d.H, static_cast<uint16_t*>(W3));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_tc(const moe_desc& d, const void* x, int T, const void* W3, float* partial, int S,
+                             int num_sms, uint32_t* flags, cudaStream_t s) {
+  CUtensorMap ma, mb;
+  cudaError_t e = make_map(&ma, W3, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)3 * d.H, (uint64_t)d.E, kBK, kBM,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e == cudaSuccess)
+    e = make_map(&mb, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.H, (uint64_t)T, kBK, kBoxRows,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  GemmArgs a{};
+  a.flags = flags;
+  a.out = partial;
+  a.R = d.E;
+  a.K = 3 * d.H;
+  a.chunk = router_tc_chunk(T);
+  a.T = T;
+  a.S = S;
+  a.Hx = d.H;
+  return launch_gemm<2, MOE_W_BF16, 1>(ma, ma, mb, a, num_sms, s);
+}
 
 // gate/up tiles 128 output rows of I (a multiple of 64; a half block is computed
 // and not stored); down tiles 128 rows of H (K = I)

@@ -50,6 +50,7 @@ struct Workspace {
   void* hbuf;         // [P, I] activations between the two projections (bf16, or fp32 for fp32 weights)
   float* yp;          // [P, H] per-pair expert outputs times routing weight, indexed by pair id
   void* xs;           // [P, H] bf16 tokens gathered in sorted order (tensor-core path)
+  void* w3;           // [E, 3H] bf16 three-way split of W_r (tensor-core router)
   size_t total;
 };
 
@@ -83,6 +84,11 @@ cudaError_t launch_gemv_gateup(const moe_desc& d, const void* x, int k, const Wo
 cudaError_t launch_gemv_down(const moe_desc& d, const float* topk_w, int k, const Workspace& ws,
                              int num_sms, uint32_t* flags, cudaStream_t s);
 bool gemm_tc_supported(const moe_desc& d);
+bool router_tc_supported(const moe_desc& d);
+int router_tc_splits(int T);
+cudaError_t launch_router_split3(const moe_desc& d, void* W3, int num_sms, cudaStream_t s);
+cudaError_t launch_router_tc(const moe_desc& d, const void* x, int T, const void* W3, float* partial, int S,
+                             int num_sms, uint32_t* flags, cudaStream_t s);
 cudaError_t launch_gather_rows(const moe_desc& d, const void* x, const Workspace& ws, int P, int num_sms,
                                cudaStream_t s);
 cudaError_t launch_gemm_gateup(const moe_desc& d, const Workspace& ws, int P, int chunk, int num_sms,

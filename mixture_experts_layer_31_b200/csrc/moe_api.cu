@@ -188,16 +188,19 @@ static int choose_path(const moe_desc& d, int32_t T) {
 
 static size_t up256(size_t v) { return (v + 255) / 256 * 256; }
 
-constexpr int kRegions = 12;
+constexpr int kRegions = 13;
 
 static void layout(const moe_desc& d, int32_t T, size_t off[kRegions], size_t* total) {
   const size_t P = (size_t)T * d.k, E = d.E;
-  const size_t S = router_splits(T);
+  const size_t S_simt = router_splits(T), S_tc = d.xfmt == MOE_X_BF16 ? router_tc_splits(T) : 0;
+  const size_t S = S_simt > S_tc ? S_simt : S_tc;
+  const size_t w3_bytes = d.xfmt == MOE_X_BF16 ? (size_t)d.E * 3 * d.H * 2 : 0;
   const size_t NC = (P + kPairChunk - 1) / kPairChunk;
   const size_t hbytes = d.wfmt == MOE_W_F32 ? 4 : 2;
   const size_t xs_bytes = (d.xfmt == MOE_X_BF16 && d.wfmt != MOE_W_F32) ? P * d.H * 2 : 0;
   const size_t sizes[kRegions] = {S * T * E * 4, (NC ? NC : 1) * E * 4, E * 4, (E + 1) * 4, (E + 1) * 4, 16 * 4,
-                                  P * 4, P * d.I * hbytes, P * d.H * 4, xs_bytes, (E + 1) * 4, (E + 1) * 4};
+                                  P * 4, P * d.I * hbytes, P * d.H * 4, xs_bytes, (E + 1) * 4, (E + 1) * 4,
+                                  w3_bytes};
   size_t o = 0;
   for (int i = 0; i < kRegions; ++i) {
     off[i] = o;
@@ -223,6 +226,7 @@ Workspace carve_workspace(const moe_desc& d, int32_t T, void* base) {
   w.xs = b + off[9];
   w.group_base = reinterpret_cast<int32_t*>(b + off[10]);
   w.tile_base = reinterpret_cast<int32_t*>(b + off[11]);
+  w.w3 = b + off[12];
   w.total = total;
   return w;
 }
@@ -267,8 +271,17 @@ extern "C" moe_status moe_route(const moe_desc* d, const void* x, int32_t T, int
   DeviceState* dev = nullptr;
   if ((st = device_state(&dev)) != MOE_OK) return st;
   const Workspace ws = carve_workspace(*d, T, workspace);
-  const int S = router_splits(T);
-  MOE_LAUNCH("router_logits", stream, launch_router_logits(*d, x, T, ws.logits, S, stream));
+  int S;
+  if (router_tc_supported(*d)) {
+    // tensor cores: fp32-accurate logits from bf16 x against the exact three-way bf16 split of W_r
+    S = router_tc_splits(T);
+    MOE_LAUNCH("router_split3", stream, launch_router_split3(*d, ws.w3, dev->num_sms, stream));
+    MOE_LAUNCH("router_logits_tc", stream,
+               launch_router_tc(*d, x, T, ws.w3, ws.logits, S, dev->num_sms, dev->flags, stream));
+  } else {
+    S = router_splits(T);
+    MOE_LAUNCH("router_logits", stream, launch_router_logits(*d, x, T, ws.logits, S, stream));
+  }
   MOE_LAUNCH("router_topk", stream, launch_router_topk(*d, ws.logits, S, T, topk_idx, topk_w, dev->flags, stream));
   return MOE_OK;
 }
