@@ -47,10 +47,8 @@ cudaError_t launch_combine(const moe_desc& d, const int32_t* idx, int T, const f
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (blocks < 1) blocks = 1;
   if (d.xfmt == MOE_X_BF16)
-    combine_kernel<true><<<blocks, 256, 0, s>>>(idx, T, d.H, d.E, d.k, yp, y);
-  else
-    combine_kernel<false><<<blocks, 256, 0, s>>>(idx, T, d.H, d.E, d.k, yp, y);
-  return cudaGetLastError();
+    return launch_k(combine_kernel<true>, dim3(blocks), dim3(256), 0, s, idx, T, d.H, d.E, d.k, yp, y);
+  return launch_k(combine_kernel<false>, dim3(blocks), dim3(256), 0, s, idx, T, d.H, d.E, d.k, yp, y);
 }
 
 }  // namespace moe

@@ -526,8 +526,7 @@ cudaError_t launch_gemm(const CUtensorMap& m0, const CUtensorMap& m1, const CUte
   auto kern = gemm_tc_kernel<MODE, WF, MT>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  kern<<<num_sms, Tr::kThreads, smem, s>>>(m0, m1, mb, a);
-  return cudaGetLastError();
+  return launch_k(kern, dim3(num_sms), dim3(Tr::kThreads), smem, s, m0, m1, mb, a);
 }
 
 // gate/up always carries two M tiles (gate, up); down carries two tiles of W_down
@@ -581,18 +580,25 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
 // relative, so bf16 x against W3 over 3H columns gives fp32-accurate logits
 __global__ void __launch_bounds__(256) split3_kernel(const float* __restrict__ Wr, int E, int H,
                                                      uint16_t* __restrict__ W3) {
-  const size_t n = (size_t)E * H;
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
-    const size_t e = i / H, h = i - e * H;
-    const float w = Wr[i];
-    const uint16_t hi = f32_to_bf16(w);
-    const float r1 = w - bf16_to_f32(hi);
-    const uint16_t mid = f32_to_bf16(r1);
-    const float r2 = r1 - bf16_to_f32(mid);
-    uint16_t* row = W3 + e * 3 * H;
-    row[h] = hi;
-    row[H + h] = mid;
-    row[2 * H + h] = f32_to_bf16(r2);
+  const int q4 = H / 4;  // float4 quads per row
+  const int n = E * q4;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const int e = i / q4, h = (i - e * q4) * 4;
+    const float4 w4 = *reinterpret_cast<const float4*>(Wr + (size_t)e * H + h);
+    const float w[4] = {w4.x, w4.y, w4.z, w4.w};
+    uint16_t p[3][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      p[0][j] = f32_to_bf16(w[j]);
+      const float r1 = w[j] - bf16_to_f32(p[0][j]);
+      p[1][j] = f32_to_bf16(r1);
+      p[2][j] = f32_to_bf16(r1 - bf16_to_f32(p[1][j]));
+    }
+    uint16_t* row = W3 + (size_t)e * 3 * H + h;
+#pragma unroll
+    for (int part = 0; part < 3; ++part)
+      *reinterpret_cast<uint2*>(row + (size_t)part * H) =
+          make_uint2((uint32_t)p[part][0] | ((uint32_t)p[part][1] << 16), (uint32_t)p[part][2] | ((uint32_t)p[part][3] << 16));
   }
 }
 
@@ -615,11 +621,10 @@ int router_tc_splits(int T) {
 bool router_tc_supported(const moe_desc& d) { return d.xfmt == MOE_X_BF16 && encode_fn() != nullptr; }
 
 cudaError_t launch_router_split3(const moe_desc& d, void* W3, int num_sms, cudaStream_t s) {
-  const size_t n = (size_t)d.E * d.H;
+  const size_t n = (size_t)d.E * d.H / 4;
   int blocks = (int)((n + 255) / 256);
-  if (blocks > num_sms * 4) blocks = num_sms * 4;
-  split3_kernel<<<blocks, 256, 0, s>>>(d.W_r, d.E, d.H, static_cast<uint16_t*>(W3));
-  return cudaGetLastError();
+  if (blocks > num_sms * 8) blocks = num_sms * 8;
+  return launch_k(split3_kernel, dim3(blocks), dim3(256), 0, s, d.W_r, d.E, d.H, static_cast<uint16_t*>(W3));
 }
 
 cudaError_t launch_router_tc(const moe_desc& d, const void* x, int T, const void* W3, float* partial, int S,
@@ -655,9 +660,9 @@ cudaError_t launch_gather_rows(const moe_desc& d, const void* x, const Workspace
   int blocks = (int)((n + 255) / 256);
   if (blocks > num_sms * 8) blocks = num_sms * 8;
   if (blocks < 1) blocks = 1;
-  gather_rows_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint16_t*>(x), d.H, d.k, ws.sorted_pair, ws.meta,
-                                            static_cast<uint16_t*>(ws.xs));
-  return cudaGetLastError();
+  return launch_k(gather_rows_kernel, dim3(blocks), dim3(256), 0, s, static_cast<const uint16_t*>(x), d.H, d.k,
+                    static_cast<const int32_t*>(ws.sorted_pair), static_cast<const int32_t*>(ws.meta),
+                    static_cast<uint16_t*>(ws.xs));
 }
 
 cudaError_t launch_gemm_gateup(const moe_desc& d, const Workspace& ws, int P, int chunk, int num_sms,

@@ -400,8 +400,7 @@ cudaError_t launch_wf(StreamArgs a, bool in_bf16, bool out_f32, int num_sms, cud
                       : (out_f32 ? gemv_stream_kernel<MODE, WF, false, true> : gemv_stream_kernel<MODE, WF, false, false>);
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  kern<<<num_sms, kThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(kern, dim3(num_sms), dim3(kThreads), smem, s, a);
 }
 
 template <int MODE>

@@ -8,6 +8,14 @@
 
 namespace moe {
 
+// Launch one kernel on stream s (plain stream ordering) and report the launch status.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                     Args&&... args) {
+  kernel<<<grid, block, smem, s>>>(static_cast<KArgs>(args)...);
+  return cudaGetLastError();
+}
+
 // Tokens are routed in chunks of this many (token, slot) pairs when building
 // the expert-sorted order.
 constexpr int kPairChunk = 1024;

@@ -230,34 +230,30 @@ bool small_sort_ok(int P, int E) { return P <= 8192 && E <= kSmallE; }
 cudaError_t launch_small_sort(const int32_t* idx, int P, int E, int chunk, int32_t* counts, int32_t* offsets,
                               int32_t* touched, int32_t* group_base, int32_t* tile_base, int32_t* meta,
                               int32_t* sorted_pair, uint32_t* flags, cudaStream_t s) {
-  small_sort_kernel<<<1, 1024, 0, s>>>(idx, P, E, chunk, counts, offsets, touched, group_base, tile_base, meta,
-                                       sorted_pair, flags);
-  return cudaGetLastError();
+  return launch_k(small_sort_kernel, dim3(1), dim3(1024), 0, s, idx, P, E, chunk, counts, offsets, touched,
+                    group_base, tile_base, meta, sorted_pair, flags);
 }
 
 cudaError_t launch_pair_histogram(const int32_t* idx, int P, int E, int32_t* chunk_hist, uint32_t* flags,
                                   cudaStream_t s) {
   const int NC = (P + kPairChunk - 1) / kPairChunk;
-  pair_histogram_kernel<<<NC, 256, E * sizeof(int32_t), s>>>(idx, P, E, chunk_hist, flags);
-  return cudaGetLastError();
+  return launch_k(pair_histogram_kernel, dim3(NC), dim3(256), E * sizeof(int32_t), s, idx, P, E, chunk_hist, flags);
 }
 
 cudaError_t launch_expert_scan(int NC, int E, int32_t* chunk_hist, int32_t* counts, int32_t* offsets,
                                int32_t* touched, int32_t* group_base, int32_t* tile_base, int chunk,
                                int32_t* meta, cudaStream_t s) {
   const int threads = ((E + 31) / 32) * 32;
-  expert_scan_kernel<<<1, threads, 0, s>>>(NC, E, chunk_hist, counts, offsets, touched, group_base, tile_base,
-                                           chunk, meta);
-  return cudaGetLastError();
+  return launch_k(expert_scan_kernel, dim3(1), dim3(threads), 0, s, NC, E, chunk_hist, counts, offsets, touched,
+                    group_base, tile_base, chunk, meta);
 }
 
 cudaError_t launch_pair_scatter(const int32_t* idx, int P, int E, const int32_t* chunk_base, int32_t* sorted_pair,
                                 cudaStream_t s) {
   const int NC = (P + kPairChunk - 1) / kPairChunk;
   const int warps = 4;
-  pair_scatter_kernel<<<(NC + warps - 1) / warps, warps * 32, warps * E * sizeof(int32_t), s>>>(
-      idx, P, E, chunk_base, sorted_pair);
-  return cudaGetLastError();
+  return launch_k(pair_scatter_kernel, dim3((NC + warps - 1) / warps), dim3(warps * 32), warps * E * sizeof(int32_t),
+                    s, idx, P, E, chunk_base, sorted_pair);
 }
 
 }  // namespace moe

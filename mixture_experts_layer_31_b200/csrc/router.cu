@@ -229,19 +229,17 @@ cudaError_t launch_router_logits(const moe_desc& d, const void* x, int T, float*
   kc = (kc + kBK - 1) / kBK * kBK;
   dim3 grid((T + kBT - 1) / kBT, (d.E + kBE - 1) / kBE, S);
   if (d.xfmt == MOE_X_BF16)
-    router_logits_kernel<true><<<grid, 256, 0, s>>>(x, d.W_r, T, d.H, d.E, kc, partial);
-  else
-    router_logits_kernel<false><<<grid, 256, 0, s>>>(x, d.W_r, T, d.H, d.E, kc, partial);
-  return cudaGetLastError();
+    return launch_k(router_logits_kernel<true>, grid, dim3(256), 0, s, x, d.W_r, T, d.H, d.E, kc, partial);
+  return launch_k(router_logits_kernel<false>, grid, dim3(256), 0, s, x, d.W_r, T, d.H, d.E, kc, partial);
 }
 
 cudaError_t launch_router_topk(const moe_desc& d, const float* partial, int S, int T, int32_t* idx,
                                float* w, uint32_t* flags, cudaStream_t s) {
   const int warps = 8;
   dim3 grid((T + warps - 1) / warps);
-#define MOE_TOPK(PL, SS)                                                                                 \
-  router_topk_kernel<PL, SS><<<grid, warps * 32, 0, s>>>(partial, T, d.E, d.k, d.router, d.b, d.expert_mask, \
-                                                         d.scale, idx, w, flags)
+#define MOE_TOPK(PL, SS)                                                                            \
+  return launch_k(router_topk_kernel<PL, SS>, grid, dim3(warps * 32), 0, s, partial, T, d.E, d.k, d.router, \
+                    d.b, d.expert_mask, d.scale, idx, w, flags)
   if (d.E <= 256) {
     switch (S) {
       case 1: MOE_TOPK(8, 1); break;
