@@ -18,8 +18,9 @@ gate/up -> down -> combine) over one batch of the workload, through the C ABI
 
 Multi-GPU: the layer does not shard on one node's hot path (one GPU, no
 sharding), so --gpus N runs N independent replicas, one per rank, each on its
-own batch ("scaling": "weak"); torch.distributed carries only the barrier and
-the max-over-ranks of the timed duration.
+own seeded batch of the workload's shape and the same layer weights
+("scaling": "weak"); torch.distributed carries only the barrier and the
+max-over-ranks of the timed duration.
 
 --impl reference runs the reference arm: the fp64 oracle (the only reference
 implementation there is) timed on the host cores, on the same workload.
@@ -296,7 +297,7 @@ def run_ours(args):
     dist_init("nccl")
     import mixture_experts_layer_31_b200 as moe
     dev = torch.device("cuda", local)
-    prob = synth.make_problem(args.config, **args.overrides)
+    prob = synth.make_problem(args.config, replica=rank, **args.overrides)
     path = {"auto": moe.MOE_PATH_AUTO, "gemv": moe.MOE_PATH_GEMV, "gemm": moe.MOE_PATH_GEMM}[args.path]
     layer = moe.MoELayer(H=prob.H, I=prob.I, E=prob.E, k=prob.k, router=prob.router, scale=prob.scale,
                          wfmt=prob.wfmt, xfmt=prob.xfmt, W_r=prob.W_r, b=prob.b, expert_mask=prob.mask,

@@ -609,12 +609,15 @@ int router_tc_chunk(int T) {
   return t < kMaxTileN ? t : kMaxTileN;
 }
 
-// K splits of the tensor-core router: a function of T only, so a masked layer and
-// its sliced twin sum identical partials in the same order
-int router_tc_splits(int T) {
+// K splits of the tensor-core router: a function of T and H only, so a masked
+// layer and its sliced twin sum identical partials in the same order.  Every
+// split owns at least one of the 3H/64 K steps (a split with none would leave
+// its TMEM accumulator unwritten).
+int router_tc_splits(int T, int H) {
   const int chunks = (T + router_tc_chunk(T) - 1) / router_tc_chunk(T);
+  const int nk_all = 3 * H / kBK;
   int S = 1;
-  while (S < 8 && chunks * S * 2 <= 74) S *= 2;
+  while (S < 8 && chunks * S * 2 <= 74 && S * 2 <= nk_all) S *= 2;
   return S;
 }
 

@@ -93,7 +93,7 @@ cudaError_t launch_gemv_down(const moe_desc& d, const float* topk_w, int k, cons
                              int num_sms, uint32_t* flags, cudaStream_t s);
 bool gemm_tc_supported(const moe_desc& d);
 bool router_tc_supported(const moe_desc& d);
-int router_tc_splits(int T);
+int router_tc_splits(int T, int H);
 cudaError_t launch_router_split3(const moe_desc& d, void* W3, int num_sms, cudaStream_t s);
 cudaError_t launch_router_tc(const moe_desc& d, const void* x, int T, const void* W3, float* partial, int S,
                              int num_sms, uint32_t* flags, cudaStream_t s);

@@ -192,7 +192,7 @@ constexpr int kRegions = 13;
 
 static void layout(const moe_desc& d, int32_t T, size_t off[kRegions], size_t* total) {
   const size_t P = (size_t)T * d.k, E = d.E;
-  const size_t S_simt = router_splits(T), S_tc = d.xfmt == MOE_X_BF16 ? router_tc_splits(T) : 0;
+  const size_t S_simt = router_splits(T), S_tc = d.xfmt == MOE_X_BF16 ? router_tc_splits(T, d.H) : 0;
   const size_t S = S_simt > S_tc ? S_simt : S_tc;
   const size_t w3_bytes = d.xfmt == MOE_X_BF16 ? (size_t)d.E * 3 * d.H * 2 : 0;
   const size_t NC = (P + kPairChunk - 1) / kPairChunk;
@@ -274,7 +274,7 @@ extern "C" moe_status moe_route(const moe_desc* d, const void* x, int32_t T, int
   int S;
   if (router_tc_supported(*d)) {
     // tensor cores: fp32-accurate logits from bf16 x against the exact three-way bf16 split of W_r
-    S = router_tc_splits(T);
+    S = router_tc_splits(T, d->H);
     MOE_LAUNCH("router_split3", stream, launch_router_split3(*d, ws.w3, dev->num_sms, stream));
     MOE_LAUNCH("router_logits_tc", stream,
                launch_router_tc(*d, x, T, ws.w3, ws.logits, S, dev->num_sms, dev->flags, stream));

@@ -248,14 +248,18 @@ def skew_bias(cfg: dict, mask: np.ndarray, c: float) -> np.ndarray:
     return b
 
 
-def make_problem(cfg_id: int, nthreads: Optional[int] = None, **overrides) -> Problem:
-    """Generate the seeded inputs of one workload (shapes may be overridden for small cases)."""
+def make_problem(cfg_id: int, nthreads: Optional[int] = None, replica: int = 0, **overrides) -> Problem:
+    """Generate the seeded inputs of one workload (shapes may be overridden for small cases).
+
+    ``replica`` r > 0 draws a different token batch x (seed + 1e6 * r) for the same
+    layer weights -- one batch per data-parallel replica."""
     c = config(cfg_id, **overrides)
     T, H, E, k, I, seed = c["T"], c["H"], c["E"], c["k"], c["I"], c["seed"]
+    x_seed = seed + 1_000_000 * int(replica)
     if c["xfmt"] == "bf16":
-        x = normal_bf16((T, H), seed, S_X, 0.0, c["x_std"], nthreads)
+        x = normal_bf16((T, H), x_seed, S_X, 0.0, c["x_std"], nthreads)
     else:
-        x = normal_f32((T, H), seed, S_X, 0.0, c["x_std"], nthreads)
+        x = normal_f32((T, H), x_seed, S_X, 0.0, c["x_std"], nthreads)
     wr_std = 1.0 / math.sqrt(H) if c["wr_std"] == "fan_in" else c["wr_std"]
     if c.get("wr_bf16"):
         W_r = bf16_bits_to_f32(normal_bf16((E, H), seed, S_WR, 0.0, wr_std, nthreads)).copy()

@@ -23,6 +23,7 @@ SMALL = {
     "kimi-bf16-ragged": (2, dict(T=45, H=256, E=32, I=192)),      # I a multiple of 64, not of 128
     "kimi-bf16-odd-H": (2, dict(T=29, H=320, E=16, I=128)),       # H not a multiple of 128: GEMV only
     "kimi-bf16-wide-E": (2, dict(T=40, H=256, E=320, I=128)),     # E > 256: wide top-k, chunked sort
+    "kimi-bf16-H64": (2, dict(T=21, H=64, E=16, k=4, I=64)),      # 3 router K steps: fewer splits than the T rule asks
     "kimi-int8-small": (3, dict(T=203, H=384, E=24, I=256)),
     "qwen3-int4-small": (4, dict(T=150, H=256, E=16, I=128)),
     "skew-masked-int8-small": (5, dict(T=301, H=256, E=40, I=128, n_active=23, bias=("skew", 0.15))),
