@@ -31,7 +31,8 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
 GATE, UP, DOWN = 0, 1, 2
-_WFMT = {"f32": 0, "bf16": 1, "int8": 2, "int4": 3}
+_WFMT = {"f32": 0, "bf16": 1, "int8": 2, "int4": 3, "int4b128": 4}
+_ACT = {"silu": 0, "gelu_tanh": 1}
 _XFMT = {"f32": 0, "bf16": 1}
 _ROUTER = {"sigmoid": 0, "softmax": 1}
 
@@ -50,7 +51,7 @@ class _Layer(ctypes.Structure):
     _fields_ = [
         ("H", ctypes.c_int32), ("I", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
         ("router", ctypes.c_int32), ("wfmt", ctypes.c_int32), ("xfmt", ctypes.c_int32),
-        ("pad", ctypes.c_int32), ("scale", ctypes.c_double),
+        ("act", ctypes.c_int32), ("scale", ctypes.c_double),
         ("W_r", ctypes.c_void_p), ("b", ctypes.c_void_p), ("mask", ctypes.c_void_p),
         ("W_gate", ctypes.c_void_p), ("W_up", ctypes.c_void_p), ("W_down", ctypes.c_void_p),
         ("s_gate", ctypes.c_void_p), ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p),
@@ -96,6 +97,7 @@ class Oracle:
         L = _Layer()
         L.H, L.I, L.E, L.k = prob.H, prob.I, prob.E, prob.k
         L.router, L.wfmt, L.xfmt = _ROUTER[prob.router], _WFMT[prob.wfmt], _XFMT[prob.xfmt]
+        L.act = _ACT[getattr(prob, "act", "silu")]
         L.scale = float(prob.scale)
         L.W_r, L.b, L.mask = _p(prob.W_r), _p(prob.b), _p(prob.mask)
         L.W_gate, L.W_up, L.W_down = _p(prob.W_gate), _p(prob.W_up), _p(prob.W_down)

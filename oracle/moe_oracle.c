@@ -25,10 +25,14 @@
  *   4. weights  w_j = r_j / sum_{selected} r * scale, with r = s (sigmoid scores,
  *               WITHOUT the bias, which only selects) or r = p (softmax).
  *   5. experts  for each selected e: g = W_gate[e] x, u = W_up[e] x,
- *               a = g * sigmoid(g) * u  (SiLU-gated), o = W_down[e] a.
+ *               a = act(g) * u  (gated), o = W_down[e] a; act = SiLU,
+ *               g * sigmoid(g), or GELU in its tanh form.
  *               "only the 8 routed experts are computed for each token" --
  *               Qwen3 card, Conversion Notes; activation 'silu' -- same card and
- *               the Kimi details page (moe op with SiLU).
+ *               the Kimi details page (moe op with SiLU); the moe op's other
+ *               activation, 'gelu_tanh', is named by the same two passages (the
+ *               runtime's error messages); its formula is the paper's, cited at
+ *               act_value below.
  *   6. combine  y[t] = sum_j w_j o_j in slot order; no residual add (the add
  *               sits outside the moe op -- Qwen3 card, Conversion Notes,
  *               moe_fusion_guard bullet).
@@ -38,14 +42,20 @@
  *   f32 / bf16 (raw 16-bit patterns) / int8 with s[E, rows] (one scale per
  *   output row and expert -- Kimi details page, quantization bullet) / int4
  *   packed two per byte, low nibble = even column, two's complement, with
- *   s[E, rows, cols/32] (block 32, fp32 scales -- Qwen3 card, Artifacts table).
+ *   s[E, rows, cols/32] (block 32, fp32 scales -- Qwen3 card, Artifacts table),
+ *   or the same nibbles with s[E, rows, cols/128] (128-wide expert blocks --
+ *   Qwen3 card, the int4 notes comparing 128-wide with 32-wide blocks).
  */
 #include <math.h>
+#ifndef M_PI
+#define M_PI 3.14159265358979323846
+#endif
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
 
-enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_INT8 = 2, ORC_INT4 = 3 };
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_INT8 = 2, ORC_INT4 = 3, ORC_INT4_B128 = 4 };
+enum { ORC_SILU = 0, ORC_GELU_TANH = 1 };
 enum { ORC_SIGMOID = 0, ORC_SOFTMAX = 1 };
 enum { ORC_GATE = 0, ORC_UP = 1, ORC_DOWN = 2 };
 
@@ -54,7 +64,7 @@ typedef struct {
   int32_t router; /* ORC_SIGMOID or ORC_SOFTMAX */
   int32_t wfmt;   /* expert storage format */
   int32_t xfmt;   /* ORC_F32 or ORC_BF16 */
-  int32_t pad;
+  int32_t act;    /* ORC_SILU or ORC_GELU_TANH */
   double scale;   /* 2.446 (Kimi) or 1 (Qwen3) */
   const float* W_r;      /* [E, H] */
   const float* b;        /* [E] or NULL (= zero bias) */
@@ -95,11 +105,13 @@ double oracle_weight(const oracle_layer* L, int which, int64_t e, int64_t row, i
       return bf16_value(((const uint16_t*)W)[r * C + col]);
     case ORC_INT8:
       return (double)((const int8_t*)W)[r * C + col] * (double)S[r];
-    case ORC_INT4: {
+    case ORC_INT4:
+    case ORC_INT4_B128: {
+      const int64_t B = L->wfmt == ORC_INT4 ? 32 : 128;
       const uint8_t byte = ((const uint8_t*)W)[r * (C / 2) + col / 2];
       int nib = (col & 1) ? (byte >> 4) : (byte & 0xF);
       if (nib >= 8) nib -= 16;
-      return (double)nib * (double)S[r * (C / 32) + col / 32];
+      return (double)nib * (double)S[r * (C / B) + col / B];
     }
   }
   return NAN;
@@ -114,6 +126,17 @@ static int count_active(const oracle_layer* L) {
 }
 
 static double sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }
+
+/* the gate's activation: SiLU g*sigmoid(g), or the tanh form of GELU,
+   g/2 * (1 + tanh(sqrt(2/pi) * (g + 0.044715 g^3))) (Hendrycks and Gimpel,
+   "Gaussian Error Linear Units", section 2) */
+static double act_value(const oracle_layer* L, double g) {
+  if (L->act == ORC_GELU_TANH) {
+    const double c = sqrt(2.0 / M_PI);
+    return 0.5 * g * (1.0 + tanh(c * (g + 0.044715 * g * g * g)));
+  }
+  return g * sigmoid(g);
+}
 
 /* ------------------------------------------------------------------ router */
 
@@ -232,7 +255,7 @@ int oracle_expert(const oracle_layer* L, int64_t e, const double* xt, double* o)
       g += oracle_weight(L, ORC_GATE, e, i, h) * xt[h];
       u += oracle_weight(L, ORC_UP, e, i, h) * xt[h];
     }
-    a[i] = g * sigmoid(g) * u;
+    a[i] = act_value(L, g) * u;
   }
   for (int64_t r = 0; r < H; ++r) {
     double acc = 0.0;

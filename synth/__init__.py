@@ -39,7 +39,9 @@ _lib = None
 # stream ids: one independent random stream per tensor
 S_X, S_WR, S_B, S_WG, S_WU, S_WD, S_MASK, S_RANK = 1, 2, 3, 4, 5, 6, 7, 8
 
-WFMT = {"f32": 0, "bf16": 1, "int8": 2, "int4": 3}
+WFMT = {"f32": 0, "bf16": 1, "int8": 2, "int4": 3, "int4b128": 4}
+ACT = {"silu": 0, "gelu_tanh": 1}
+INT4_BLOCK = {"int4": 32, "int4b128": 128}
 XFMT = {"f32": 0, "bf16": 1}
 ROUTER = {"sigmoid": 0, "softmax": 1}
 
@@ -67,6 +69,7 @@ def _load():
             "synth_uniform_f64": [vp, sz, u64, u64, dbl, dbl],
             "synth_int8_rows": [vp, vp, sz, sz, u64, u64, dbl, i32],
             "synth_int4_blocks": [vp, vp, sz, sz, u64, u64, dbl, i32],
+            "synth_int4_blocks_b": [vp, vp, sz, sz, sz, u64, u64, dbl, i32],
         }.items():
             f = getattr(lib, name)
             f.argtypes = args
@@ -119,11 +122,12 @@ def int8_rows(rows, cols, seed, stream, std, nthreads=None):
     return q, s
 
 
-def int4_blocks(rows, cols, seed, stream, std, nthreads=None):
-    """N(0, std) matrix [rows, cols] stored as int4 nibbles [rows, cols/2] + scales [rows, cols/32]."""
+def int4_blocks(rows, cols, seed, stream, std, nthreads=None, block=32):
+    """N(0, std) matrix [rows, cols] stored as int4 nibbles [rows, cols/2] + scales [rows, cols/block]."""
     q = np.empty((rows, cols // 2), np.uint8)
-    s = np.empty((rows, cols // 32), np.float32)
-    assert _load().synth_int4_blocks(_ptr(q), _ptr(s), rows, cols, seed, stream, std, _threads(nthreads)) == 0
+    s = np.empty((rows, cols // block), np.float32)
+    assert _load().synth_int4_blocks_b(_ptr(q), _ptr(s), rows, cols, block, seed, stream, std,
+                                       _threads(nthreads)) == 0
     return q, s
 
 
@@ -191,7 +195,8 @@ class Problem:
     W_down: np.ndarray       # [E,H,I] (int4: [E,H,I/2] uint8)
     s_gate: Optional[np.ndarray] = None  # int8 [E,I]; int4 [E,I,H/32]
     s_up: Optional[np.ndarray] = None
-    s_down: Optional[np.ndarray] = None  # int8 [E,H]; int4 [E,H,I/32]
+    s_down: Optional[np.ndarray] = None  # int8 [E,H]; int4 [E,H,I/32] (int4b128: I/128)
+    act: str = "silu"                    # gated activation: "silu" or "gelu_tanh"
 
     def weight_bytes_per_expert(self) -> int:
         n = 0
@@ -211,9 +216,10 @@ def _expert_weights(fmt, E, rows, cols, seed, stream, std, nthreads):
     if fmt == "int8":
         q, s = int8_rows(E * rows, cols, seed, stream, std, nthreads)
         return q.reshape(E, rows, cols), s.reshape(E, rows)
-    if fmt == "int4":
-        q, s = int4_blocks(E * rows, cols, seed, stream, std, nthreads)
-        return q.reshape(E, rows, cols // 2), s.reshape(E, rows, cols // 32)
+    if fmt in INT4_BLOCK:
+        B = INT4_BLOCK[fmt]
+        q, s = int4_blocks(E * rows, cols, seed, stream, std, nthreads, block=B)
+        return q.reshape(E, rows, cols // 2), s.reshape(E, rows, cols // B)
     raise ValueError(fmt)
 
 
@@ -285,4 +291,4 @@ def make_problem(cfg_id: int, nthreads: Optional[int] = None, replica: int = 0, 
     return Problem(cfg=c, T=T, H=H, I=I, E=E, k=k, router=c["router"], scale=float(c["scale"]),
                    wfmt=c["wfmt"], xfmt=c["xfmt"], x=x, W_r=W_r, b=b, mask=mask,
                    W_gate=W_gate, W_up=W_up, W_down=W_down,
-                   s_gate=s_gate, s_up=s_up, s_down=s_down)
+                   s_gate=s_gate, s_up=s_up, s_down=s_down, act=c.get("act", "silu"))

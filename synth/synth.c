@@ -108,6 +108,7 @@ struct job {
   uint64_t key;
   double a, b;
   size_t rows, cols;
+  size_t block; /* int4: quantisation block along the columns (32 or 128) */
 };
 
 typedef struct {
@@ -213,15 +214,15 @@ static void fill_int8_rows(const job* j, size_t lo, size_t hi) {
 static void fill_int4_blocks(const job* j, size_t lo, size_t hi) {
   uint8_t* q = (uint8_t*)j->out;
   float* s = (float*)j->out2;
-  const size_t C = j->cols, NB = C / 32;
+  const size_t B = j->block, C = j->cols, NB = C / B;
   const double floor_scale = 1.0 / 16384.0; /* 2^-14 */
-  float w[32];
-  double z[32];
+  float w[128];
+  double z[128];
   for (size_t r = lo; r < hi; ++r) {
     for (size_t bi = 0; bi < NB; ++bi) {
       double amax = 0.0;
-      normal_range(j->key, r * C + bi * 32, r * C + bi * 32 + 32, z);
-      for (size_t c = 0; c < 32; ++c) {
+      normal_range(j->key, r * C + bi * B, r * C + bi * B + B, z);
+      for (size_t c = 0; c < B; ++c) {
         w[c] = (float)(j->b * z[c]);
         const double a = fabs((double)w[c]);
         if (a > amax) amax = a;
@@ -231,7 +232,7 @@ static void fill_int4_blocks(const job* j, size_t lo, size_t hi) {
       float sc = (float)scd;
       if ((double)sc < floor_scale) sc = (float)floor_scale;
       s[r * NB + bi] = sc;
-      for (size_t c = 0; c < 32; c += 2) {
+      for (size_t c = 0; c < B; c += 2) {
         int v[2];
         for (int h = 0; h < 2; ++h) {
           double t = round_half_away((double)w[c + h] / (double)sc);
@@ -239,7 +240,7 @@ static void fill_int4_blocks(const job* j, size_t lo, size_t hi) {
           if (t < -8.0) t = -8.0;
           v[h] = (int)t;
         }
-        q[r * (C / 2) + (bi * 32 + c) / 2] = (uint8_t)((v[0] & 0xF) | ((v[1] & 0xF) << 4));
+        q[r * (C / 2) + (bi * B + c) / 2] = (uint8_t)((v[0] & 0xF) | ((v[1] & 0xF) << 4));
       }
     }
   }
@@ -288,13 +289,19 @@ int synth_int8_rows(int8_t* q, float* s, size_t rows, size_t cols, uint64_t seed
   return 0;
 }
 
-/* q: [rows, cols/2] packed nibbles, s: [rows, cols/32] fp32; cols % 32 == 0 */
-int synth_int4_blocks(uint8_t* q, float* s, size_t rows, size_t cols, uint64_t seed, uint64_t stream,
-                      double std, int nthreads) {
-  if (((!q || !s) && rows) || cols % 32) return -1;
-  job j = {fill_int4_blocks, q, s, stream_key(seed, stream), 0.0, std, rows, cols};
+/* q: [rows, cols/2] packed nibbles, s: [rows, cols/block] fp32; block 32 or 128,
+   cols % block == 0.  The real-valued weights do not depend on the block size. */
+int synth_int4_blocks_b(uint8_t* q, float* s, size_t rows, size_t cols, size_t block, uint64_t seed,
+                        uint64_t stream, double std, int nthreads) {
+  if (((!q || !s) && rows) || (block != 32 && block != 128) || cols % block) return -1;
+  job j = {fill_int4_blocks, q, s, stream_key(seed, stream), 0.0, std, rows, cols, block};
   fan_out(&j, rows, nthreads);
   return 0;
+}
+
+int synth_int4_blocks(uint8_t* q, float* s, size_t rows, size_t cols, uint64_t seed, uint64_t stream,
+                      double std, int nthreads) {
+  return synth_int4_blocks_b(q, s, rows, cols, 32, seed, stream, std, nthreads);
 }
 
 /* raw stream access, for checking the generator itself */

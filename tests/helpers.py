@@ -36,7 +36,8 @@ def dense_weights(prob, which):
         return synth.bf16_bits_to_f32(W).astype(np.float64)
     if prob.wfmt == "int8":
         return W.astype(np.float64) * S[..., None].astype(np.float64)
-    if prob.wfmt == "int4":
+    if prob.wfmt in ("int4", "int4b128"):
+        block = 32 if prob.wfmt == "int4" else 128
         lo = (W & 0xF).astype(np.int64)
         hi = (W >> 4).astype(np.int64)
         lo = np.where(lo >= 8, lo - 16, lo)
@@ -44,7 +45,7 @@ def dense_weights(prob, which):
         q = np.empty(W.shape[:-1] + (W.shape[-1] * 2,), np.float64)
         q[..., 0::2] = lo
         q[..., 1::2] = hi
-        return q * np.repeat(S.astype(np.float64), 32, axis=-1)
+        return q * np.repeat(S.astype(np.float64), block, axis=-1)
     raise ValueError(prob.wfmt)
 
 
@@ -54,11 +55,13 @@ def dense_x(prob):
     return prob.x.astype(np.float64)
 
 
-def textbook_swiglu(x, Wg, Wu, Wd):
-    """torch library SwiGLU FFN in fp64: Wd (silu(Wg x) * (Wu x)) for rows of x."""
+def textbook_swiglu(x, Wg, Wu, Wd, act="silu"):
+    """torch library gated FFN in fp64: Wd (act(Wg x) * (Wu x)) for rows of x, with act
+    torch's silu or its tanh-approximated gelu."""
     x = torch.as_tensor(x, dtype=torch.float64)
-    return F.linear(F.silu(F.linear(x, torch.as_tensor(Wg))) * F.linear(x, torch.as_tensor(Wu)),
-                    torch.as_tensor(Wd)).numpy()
+    g = F.linear(x, torch.as_tensor(Wg))
+    a = F.silu(g) if act == "silu" else F.gelu(g, approximate="tanh")
+    return F.linear(a * F.linear(x, torch.as_tensor(Wu)), torch.as_tensor(Wd)).numpy()
 
 
 def ln_expr(s: str) -> float:

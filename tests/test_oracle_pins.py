@@ -110,18 +110,32 @@ def test_k1_weight_is_scale():
     assert (w == np.float64(2.446)).all()
 
 
-@pytest.mark.parametrize("wfmt", ["f32", "bf16", "int8", "int4"])
+@pytest.mark.parametrize("act", ["silu", "gelu_tanh"])
+@pytest.mark.parametrize("wfmt", ["f32", "bf16", "int8", "int4", "int4b128"])
 @pytest.mark.parametrize("xfmt", ["f32", "bf16"])
-def test_single_expert_reduces_to_dense_swiglu(wfmt, xfmt):
-    """k = E = 1: the layer is scale * SwiGLU(x), checked against torch's silu/linear
-    on independently decoded weights, for every stored weight format."""
-    prob = synth.make_problem(1, T=5, H=64, I=64, E=1, k=1, wfmt=wfmt, xfmt=xfmt, seed=77,
-                              w_std=0.05, bias=None)
+def test_single_expert_reduces_to_dense_swiglu(wfmt, xfmt, act):
+    """k = E = 1: the layer is scale * act(W_gate x) * (W_up x) through W_down, checked
+    against torch's silu / tanh-gelu and linear on independently decoded weights, for
+    every stored weight format and both activations."""
+    n = 128 if wfmt == "int4b128" else 64
+    prob = synth.make_problem(1, T=5, H=n, I=n, E=1, k=1, wfmt=wfmt, xfmt=xfmt, seed=77,
+                              w_std=0.05, bias=None, act=act)
     y, idx, w, _ = oracle.Oracle(prob).forward()
     assert (idx == 0).all()
     ref = prob.scale * textbook_swiglu(dense_x(prob), dense_weights(prob, "gate")[0],
-                                       dense_weights(prob, "up")[0], dense_weights(prob, "down")[0])
+                                       dense_weights(prob, "up")[0], dense_weights(prob, "down")[0], act)
     np.testing.assert_allclose(y, ref, rtol=1e-11, atol=1e-12)
+
+
+def test_activations_differ_where_they_should():
+    """The activation attribute reaches the expert: SiLU and tanh-GELU give different
+    outputs on the same layer, and both vanish with the gate weights."""
+    a = synth.make_problem(1, T=3, H=64, I=64, E=4, k=2, seed=78)
+    b = synth.make_problem(1, T=3, H=64, I=64, E=4, k=2, seed=78, act="gelu_tanh")
+    ya, ia, _, _ = oracle.Oracle(a, nthreads=1).forward()
+    yb, ib, _, _ = oracle.Oracle(b, nthreads=1).forward()
+    assert (ia == ib).all()
+    assert np.abs(ya - yb).max() > 1e-3 * np.abs(ya).max()
 
 
 @pytest.mark.parametrize("router", ["sigmoid", "softmax"])
@@ -210,12 +224,12 @@ def test_softmax_denominator_cancels():
         np.testing.assert_allclose(w[t], scipy.special.softmax(logits[t][idx[t]]), rtol=1e-12)
 
 
-@pytest.mark.parametrize("wfmt", ["int8", "int4", "bf16"])
+@pytest.mark.parametrize("wfmt", ["int8", "int4", "int4b128", "bf16"])
 def test_oracle_dequantisation_matches_real_weights(wfmt):
     """The oracle's decode of each stored format lies within half a quantisation step
     of the real-valued weight the encoder started from (regenerated from the same
     random stream); bf16 within half an ulp."""
-    H, I, E = 64, 96, 3
+    H, I, E = (128, 256, 3) if wfmt == "int4b128" else (64, 96, 3)
     prob = synth.make_problem(3, T=2, H=H, I=I, E=E, wfmt=wfmt, seed=5)
     orc = oracle.Oracle(prob, nthreads=1)
     for which, name, rows, cols in ((0, "gate", I, H), (2, "down", H, I)):
@@ -229,8 +243,8 @@ def test_oracle_dequantisation_matches_real_weights(wfmt):
                 s = float(getattr(prob, "s_" + name)[e, r])
                 assert abs(v - real[e, r, c]) <= s / 2 * (1 + 1e-6)
                 assert abs(v / s - round(v / s)) < 1e-9 and abs(v / s) <= 127
-            elif wfmt == "int4":
-                s = float(getattr(prob, "s_" + name)[e, r, c // 32])
+            elif wfmt in ("int4", "int4b128"):
+                s = float(getattr(prob, "s_" + name)[e, r, c // (32 if wfmt == "int4" else 128)])
                 assert s >= 2.0 ** -14
                 assert abs(v - real[e, r, c]) <= s / 2 * (1 + 1e-6)
                 assert -8 <= round(v / s) <= 7
