@@ -72,8 +72,11 @@ def _load():
         lib.oracle_expert.argtypes = [P, i64, vp, vp]
         lib.oracle_combine.argtypes = [P, vp, i64, i64, vp, vp, vp]
         lib.oracle_forward.argtypes = [P, vp, i64, i64, vp, vp, vp, vp]
+        lib.oracle_expert_counts.argtypes = [vp, i64, ctypes.c_int32, vp]
+        lib.oracle_cover_set.argtypes = [vp, ctypes.c_int32, ctypes.c_double, vp, vp, vp]
         for f in ("oracle_router_logits", "oracle_keys", "oracle_select", "oracle_route",
-                  "oracle_expert", "oracle_combine", "oracle_forward"):
+                  "oracle_expert", "oracle_combine", "oracle_forward", "oracle_expert_counts",
+                  "oracle_cover_set"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -204,3 +207,28 @@ class Oracle:
         tokens = list(range(self.prob.T)) if tokens is None else [int(t) for t in tokens]
         idx, w, margin = self.route(tokens)
         return self.combine(tokens, idx, w), idx, w, margin
+
+
+# -- routing statistics (CMF code specialist page, How it was made: Calibrate and Defrag) --
+
+def expert_counts(idx: np.ndarray, E: int, counts: Optional[np.ndarray] = None) -> np.ndarray:
+    """counts[e] += number of routing entries equal to e (entries outside [0, E) skipped)."""
+    idx = np.ascontiguousarray(idx, np.int32)
+    counts = np.zeros(E, np.uint64) if counts is None else counts
+    assert counts.dtype == np.uint64 and counts.flags["C_CONTIGUOUS"] and counts.size == E
+    assert _load().oracle_expert_counts(_p(idx), idx.size, int(E), _p(counts)) == 0
+    return counts
+
+
+def cover_set(counts: np.ndarray, cover: float):
+    """(keep [E] uint8, new_index [E] int32, n_keep): the smallest expert set whose
+    counts reach cover * total, renumbered into a dense prefix."""
+    counts = np.ascontiguousarray(counts, np.uint64)
+    E = counts.size
+    keep = np.empty(E, np.uint8)
+    new_index = np.empty(E, np.int32)
+    n = np.empty(1, np.int32)
+    rc = _load().oracle_cover_set(_p(counts), int(E), float(cover), _p(keep), _p(new_index), _p(n))
+    if rc != 0:
+        raise ValueError("oracle_cover_set rejected its arguments")
+    return keep, new_index, int(n[0])

@@ -303,3 +303,52 @@ int oracle_forward(const oracle_layer* L, const void* x, int64_t t0, int64_t t1,
   if (rc == 0) rc = oracle_combine(L, x, t0, t1, idx, w, y);
   return rc;
 }
+
+/* ------------------------------------------------------- routing statistics */
+/*
+ * Per-expert routing frequencies and the covering expert set (CMF code
+ * specialist page, How it was made: the Calibrate step records per-layer expert
+ * routing frequencies over a corpus; the Defrag step keeps, per layer, the
+ * smallest expert set that covers a given share (0.95) of that routing mass,
+ * renumbers the kept experts into a dense prefix and slices router rows and
+ * selection bias to match).
+ */
+
+/* counts[e] += number of (token, slot) entries equal to e; entries outside
+   [0, E) are not counted */
+int oracle_expert_counts(const int32_t* idx, int64_t n, int32_t E, uint64_t* counts) {
+  if ((!idx && n) || !counts || E < 1 || n < 0) return -1;
+  for (int64_t i = 0; i < n; ++i)
+    if (idx[i] >= 0 && idx[i] < E) counts[idx[i]] += 1;
+  return 0;
+}
+
+/*
+ * Smallest set of experts whose counts reach cover * (sum of counts): experts
+ * are taken by count descending (ties: lower index first) until the running
+ * sum, as a double, is >= cover * total.  keep[e] = 1 for kept experts;
+ * new_index[e] = position of e among the kept experts in ascending index order
+ * (the dense prefix), or -1.  cover must lie in (0, 1].
+ */
+int oracle_cover_set(const uint64_t* counts, int32_t E, double cover, uint8_t* keep, int32_t* new_index,
+                     int32_t* n_keep) {
+  if (!counts || !keep || !new_index || !n_keep || E < 1 || !(cover > 0.0 && cover <= 1.0)) return -1;
+  uint64_t total = 0;
+  for (int e = 0; e < E; ++e) total += counts[e];
+  const double target = cover * (double)total;
+  for (int e = 0; e < E; ++e) keep[e] = 0;
+  uint64_t cum = 0;
+  int taken = 0;
+  while ((double)cum < target && taken < E) {
+    int best = -1; /* the largest count not yet kept, lowest index on ties */
+    for (int e = 0; e < E; ++e)
+      if (!keep[e] && (best < 0 || counts[e] > counts[best])) best = e;
+    keep[best] = 1;
+    cum += counts[best];
+    ++taken;
+  }
+  int next = 0;
+  for (int e = 0; e < E; ++e) new_index[e] = keep[e] ? next++ : -1;
+  *n_keep = taken;
+  return 0;
+}
