@@ -245,7 +245,7 @@ def time_oracle(prob, budget_s: float, max_tokens=None):
 
 def config_block(prob, cid, extra=None):
     c = {"workload": prob.cfg["workload"], "T": prob.T, "H": prob.H, "E": prob.E, "k": prob.k, "I": prob.I,
-         "experts": prob.wfmt, "activations": prob.xfmt, "router": prob.router,
+         "experts": prob.wfmt, "activations": prob.xfmt, "router": prob.router, "act": prob.act,
          "active_experts": int(prob.mask.sum()) if prob.mask is not None else prob.E,
          "l2": "flushed between steps (512 MB write, outside timed intervals); expert weights >> L2",
          "parallelism": "replicas"}
@@ -302,7 +302,7 @@ def run_ours(args):
     layer = moe.MoELayer(H=prob.H, I=prob.I, E=prob.E, k=prob.k, router=prob.router, scale=prob.scale,
                          wfmt=prob.wfmt, xfmt=prob.xfmt, W_r=prob.W_r, b=prob.b, expert_mask=prob.mask,
                          W_gate=prob.W_gate, W_up=prob.W_up, W_down=prob.W_down, s_gate=prob.s_gate,
-                         s_up=prob.s_up, s_down=prob.s_down, path=path, device=dev)
+                         s_up=prob.s_up, s_down=prob.s_down, path=path, device=dev, act=prob.act)
     if prob.xfmt == "bf16":
         x_host = torch.from_numpy(prob.x.view(np.int16)).view(torch.bfloat16)
     else:

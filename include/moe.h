@@ -75,15 +75,20 @@ typedef enum {
   MOE_W_F32 = 0,
   MOE_W_BF16 = 1,
   MOE_W_INT8_ROW = 2, /* int8, one fp32 scale per (expert, output row) */
-  MOE_W_INT4_B32 = 3  /* int4 two's complement, 2 per byte (low nibble = even
+  MOE_W_INT4_B32 = 3, /* int4 two's complement, 2 per byte (low nibble = even
                          column), one fp32 scale per 32 columns */
+  MOE_W_INT4_B128 = 4 /* the same nibbles, one fp32 scale per 128 columns (the
+                         128-wide expert blocks of the Qwen3-30B-A3B LiteRT-LM
+                         card's int4 notes); H and I multiples of 128 */
 } moe_wfmt;
 
 typedef enum { MOE_X_F32 = 0, MOE_X_BF16 = 1 } moe_xfmt;
 
 typedef enum {
-  MOE_ACT_SILU = 0,
-  MOE_ACT_GELU_TANH = 1 /* named by the pages' moe op; rejected with MOE_ERR_UNSUPPORTED */
+  MOE_ACT_SILU = 0,     /* h = g * sigmoid(g) * u */
+  MOE_ACT_GELU_TANH = 1 /* h = g/2 * (1 + tanh(sqrt(2/pi) (g + 0.044715 g^3))) * u: the
+                           moe op's other activation, 'gelu_tanh' (Kimi-Linear details
+                           page, Runtime; Qwen3 card, Conversion Notes) */
 } moe_act;
 
 typedef enum {
@@ -97,9 +102,10 @@ typedef enum {
  * (zero bias); expert_mask [E] uint8 (1 = active) or NULL (all active).
  *   W_gate, W_up : [E, I, H]   (int4: [E, I, H/2] bytes)
  *   W_down       : [E, H, I]   (int4: [E, H, I/2] bytes)
- *   s_gate, s_up : int8 [E, I];  int4 [E, I, H/32];  otherwise NULL
- *   s_down       : int8 [E, H];  int4 [E, H, I/32];  otherwise NULL
- * Limits: H, I multiples of 64; 1 <= k <= 32; k <= E <= 1024.
+ *   s_gate, s_up : int8 [E, I];  int4 [E, I, H/32] (block 128: H/128);  otherwise NULL
+ *   s_down       : int8 [E, H];  int4 [E, H, I/32] (block 128: I/128);  otherwise NULL
+ * Limits: H, I multiples of 64 (of 128 for int4 block 128); 1 <= k <= 32;
+ * k <= E <= 1024.
  */
 typedef struct {
   int32_t H, I, E, k;
@@ -171,6 +177,34 @@ MOE_API moe_status moe_forward(const moe_desc* d, const void* x, int32_t T, cons
 #define MOE_NOALLOC_SCRATCH_BYTES (16u << 20)
 MOE_API moe_status moe_forward_noalloc(const moe_desc* d, const void* x, int32_t T, const int32_t* topk_idx,
                                        const float* topk_w, void* y, cudaStream_t stream);
+
+/*
+ * Routing statistics (CMF code specialist page, How it was made: Calibrate and
+ * Defrag steps).
+ *
+ * moe_expert_counts: per-expert routing frequencies, accumulated across calls.
+ *   topk_idx [T, k] int32 (device; routing from moe_route or the caller),
+ *   counts [E] uint64 (device, caller-owned and zeroed once by the caller; each
+ *   call adds, for every expert e, the number of entries of topk_idx equal to
+ *   e).  Entries outside [0, E) are skipped, not flagged.  Only d->E and d->k
+ *   are read from the descriptor.  Asynchronous on `stream`.  The adds are
+ *   integer atomics, so calls adding into the same counts from several streams
+ *   give the exact total in any order.
+ *
+ * moe_cover_set: host utility for the Defrag step.  counts [E] (HOST memory),
+ *   cover in (0, 1].  Keeps the smallest set of experts whose counts reach
+ *   cover * (sum of counts), taking experts by count descending with ties to
+ *   the lower index.  Writes keep [E] (HOST, 1 = kept: usable directly as
+ *   moe_desc.expert_mask once copied to the device), new_index [E] (HOST, the
+ *   kept expert's position in the dense prefix that keeps the original index
+ *   order, -1 for dropped experts; router rows, selection bias and experts are
+ *   sliced in this order) and *n_keep.  All-zero counts keep no expert.
+ *   Synchronous, no device work.
+ */
+MOE_API moe_status moe_expert_counts(const moe_desc* d, const int32_t* topk_idx, int32_t T, uint64_t* counts,
+                                     cudaStream_t stream);
+MOE_API moe_status moe_cover_set(const uint64_t* counts, int32_t E, double cover, uint8_t* keep,
+                                 int32_t* new_index, int32_t* n_keep);
 
 /* Message for the last non-OK status returned on this thread ("" if none). */
 MOE_API const char* moe_last_error(void);

@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 # enums (mirror include/moe.h)
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA = 0, 1, 2, 3, 4
 MOE_ROUTER_SIGMOID_BIAS, MOE_ROUTER_SOFTMAX = 0, 1
-MOE_W_F32, MOE_W_BF16, MOE_W_INT8_ROW, MOE_W_INT4_B32 = 0, 1, 2, 3
+MOE_W_F32, MOE_W_BF16, MOE_W_INT8_ROW, MOE_W_INT4_B32, MOE_W_INT4_B128 = 0, 1, 2, 3, 4
 MOE_X_F32, MOE_X_BF16 = 0, 1
 MOE_ACT_SILU, MOE_ACT_GELU_TANH = 0, 1
 MOE_PATH_AUTO, MOE_PATH_GEMV, MOE_PATH_GEMM = 0, 1, 2
@@ -30,12 +30,15 @@ MOE_FLAG_BAD_EXPERT_INDEX, MOE_FLAG_TOO_FEW_ACTIVE, MOE_FLAG_NONFINITE_LOGIT = 1
 
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
                 4: "MOE_ERR_CUDA"}
-WFMT = {"f32": MOE_W_F32, "bf16": MOE_W_BF16, "int8": MOE_W_INT8_ROW, "int4": MOE_W_INT4_B32}
+WFMT = {"f32": MOE_W_F32, "bf16": MOE_W_BF16, "int8": MOE_W_INT8_ROW, "int4": MOE_W_INT4_B32,
+        "int4b128": MOE_W_INT4_B128}
+ACT = {"silu": MOE_ACT_SILU, "gelu_tanh": MOE_ACT_GELU_TANH}
 XFMT = {"f32": MOE_X_F32, "bf16": MOE_X_BF16}
 ROUTER = {"sigmoid": MOE_ROUTER_SIGMOID_BIAS, "softmax": MOE_ROUTER_SOFTMAX}
 
-EXPORTS = ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_noalloc", "moe_last_error",
-           "moe_device_flags", "moe_launch_count", "moe_stage_timing", "moe_stage_times")
+EXPORTS = ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_noalloc", "moe_expert_counts",
+           "moe_cover_set", "moe_last_error", "moe_device_flags", "moe_launch_count", "moe_stage_timing",
+           "moe_stage_times")
 MOE_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -71,6 +74,8 @@ def _load() -> ctypes.CDLL:
     lib.moe_route.argtypes = [D, vp, i32, vp, vp, vp, sz, vp]
     lib.moe_forward.argtypes = [D, vp, i32, vp, vp, vp, vp, sz, vp]
     lib.moe_forward_noalloc.argtypes = [D, vp, i32, vp, vp, vp, vp]
+    lib.moe_expert_counts.argtypes = [D, vp, i32, vp, vp]
+    lib.moe_cover_set.argtypes = [vp, i32, ctypes.c_double, vp, vp, ctypes.POINTER(i32)]
     lib.moe_last_error.argtypes = []
     lib.moe_last_error.restype = ctypes.c_char_p
     lib.moe_device_flags.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
@@ -78,8 +83,8 @@ def _load() -> ctypes.CDLL:
     lib.moe_launch_count.restype = ctypes.c_uint64
     lib.moe_stage_timing.argtypes = [i32]
     lib.moe_stage_times.argtypes = [ctypes.POINTER(moe_stage_time), i32, ctypes.POINTER(i32)]
-    for f in ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_noalloc", "moe_device_flags",
-              "moe_stage_timing", "moe_stage_times"):
+    for f in ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_noalloc", "moe_expert_counts",
+              "moe_cover_set", "moe_device_flags", "moe_stage_timing", "moe_stage_times"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -125,6 +130,25 @@ def moe_forward_noalloc(desc: moe_desc, x: int, T: int, topk_idx: int, topk_w: i
     _check(lib().moe_forward_noalloc(ctypes.byref(desc), x, int(T), topk_idx, topk_w, y, stream))
 
 
+def moe_expert_counts(desc: moe_desc, topk_idx: int, T: int, counts: int, stream: int = 0) -> None:
+    """counts[e] (device uint64 [E]) += entries of topk_idx [T, k] equal to e."""
+    _check(lib().moe_expert_counts(ctypes.byref(desc), topk_idx, int(T), counts, stream))
+
+
+def moe_cover_set(counts, cover: float):
+    """Host utility: (keep [E] uint8, new_index [E] int32, n_keep) for the smallest
+    expert set whose counts (host array [E]) reach cover * total."""
+    import numpy as np
+    c = np.ascontiguousarray(counts, dtype=np.uint64)
+    E = c.size
+    keep = np.empty(E, np.uint8)
+    new_index = np.empty(E, np.int32)
+    n = ctypes.c_int32(0)
+    _check(lib().moe_cover_set(c.ctypes.data, int(E), float(cover), keep.ctypes.data, new_index.ctypes.data,
+                               ctypes.byref(n)))
+    return keep, new_index, int(n.value)
+
+
 def moe_last_error() -> str:
     return lib().moe_last_error().decode()
 
@@ -159,7 +183,8 @@ class MoELayer:
     workspace, and calls moe_route / moe_forward on the current torch stream."""
 
     def __init__(self, *, H, I, E, k, router, scale, wfmt, xfmt, W_r, W_gate, W_up, W_down, b=None,
-                 expert_mask=None, s_gate=None, s_up=None, s_down=None, path=MOE_PATH_AUTO, device="cuda"):
+                 expert_mask=None, s_gate=None, s_up=None, s_down=None, path=MOE_PATH_AUTO, device="cuda",
+                 act="silu"):
         import torch
         lib()  # fail loudly now if the CUDA library is missing
         self.torch = torch
@@ -182,7 +207,7 @@ class MoELayer:
         d = moe_desc()
         d.H, d.I, d.E, d.k = int(H), int(I), int(E), int(k)
         d.router = ROUTER[router] if isinstance(router, str) else int(router)
-        d.act = MOE_ACT_SILU
+        d.act = ACT[act] if isinstance(act, str) else int(act)
         d.wfmt = WFMT[wfmt] if isinstance(wfmt, str) else int(wfmt)
         d.xfmt = XFMT[xfmt] if isinstance(xfmt, str) else int(xfmt)
         d.path = int(path)
@@ -230,3 +255,11 @@ class MoELayer:
     def __call__(self, x):
         idx, w = self.route(x)
         return self.forward(x, idx, w), idx, w
+
+    def expert_counts(self, idx, counts=None):
+        """Accumulate per-expert routing counts of idx [T, k] into counts (a device
+        uint64 tensor [E], created zeroed when None) and return it."""
+        if counts is None:
+            counts = self.torch.zeros(self.desc.E, dtype=self.torch.uint64, device=self.device)
+        moe_expert_counts(self.desc, idx.data_ptr(), idx.shape[0], counts.data_ptr(), self._stream())
+        return counts

@@ -33,6 +33,18 @@ __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f +
 // The same with CUDA's fast intrinsics (a few ulp), for outputs rounded to bf16
 // afterwards.  The exponent argument is capped so 1 + e stays below 2^126, the
 // range where __fdividef is exact to its stated error.
+// tanh-form GELU of the gate times up.  (1 + tanh z) / 2 = 1 / (1 + exp(-2z)),
+// so gelu(g) = g / (1 + exp(-2z)) with z = sqrt(2/pi) (g + 0.044715 g^3).
+__device__ __forceinline__ float gelu_tanh_z(float g) {
+  return 0.7978845608028654f * fmaf(0.044715f * g, g * g, g);
+}
+__device__ __forceinline__ float gelu_tanh_mul(float g, float u) {
+  return g / (1.0f + expf(-2.0f * gelu_tanh_z(g))) * u;
+}
+__device__ __forceinline__ float gelu_tanh_mul_fast(float g, float u) {
+  return __fdividef(g, 1.0f + __expf(fminf(-2.0f * gelu_tanh_z(g), 80.0f))) * u;
+}
+
 __device__ __forceinline__ float silu_mul_fast(float g, float u) {
   return __fdividef(g, 1.0f + __expf(fminf(-g, 80.0f))) * u;
 }

@@ -45,7 +45,7 @@ constexpr int kBarrierBytes = 1024;
 constexpr int kSmemLimit = 232448;         // 227 KB opt-in
 
 struct GemmArgs {
-  const float* s0;  // scales of W0 (int8: [E,R]; int4: [E,R,K/32])
+  const float* s0;  // scales of W0 (int8: [E,R]; int4: [E,R,K >> qsh])
   const float* s1;  // scales of W1 (gate/up)
   const int32_t* offsets;
   const int32_t* touched;
@@ -69,6 +69,8 @@ struct GemmArgs {
   int T;
   int S;
   int Hx;               // columns of x (the K coordinate of x is taken modulo Hx)
+  int act;              // gate/up: moe_act (SiLU or tanh-GELU)
+  int qsh;              // int4: log2 of the scale block (5: 32 columns, 7: 128)
 };
 
 __device__ __forceinline__ void wait_or_die(uint64_t* bar, uint32_t parity, bool& dead, uint32_t* flags) {
@@ -345,7 +347,8 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
                 if (n0 + j < t.n_tok) {
-                  const float hv = silu_mul_fast(__uint_as_float(g[j]) * sg, __uint_as_float(v[j]) * su);
+                  const float gv = __uint_as_float(g[j]) * sg, uv = __uint_as_float(v[j]) * su;
+                  const float hv = a.act == MOE_ACT_GELU_TANH ? gelu_tanh_mul_fast(gv, uv) : silu_mul_fast(gv, uv);
                   hout[(size_t)(pos0 + n0 + j) * a.R + row] = f32_to_bf16(hv);
                 }
               }
@@ -418,15 +421,16 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
         const float* S = (MODE == 0 && mt == 1) ? a.s1 : a.s0;
         int wr = MODE == 0 ? t.ib * kBM + rr : t.ib * Tr::kRows + mt * kBM + rr;
         if (wr >= a.R) wr = a.R - 1;  // rows past a half block are computed but never stored
-        srow[j] = S + ((size_t)t.e * a.R + wr) * (a.K / 32) + (c8 >> 2);
-        sc_next[j] = WF == MOE_W_INT4_B32 ? __ldg(srow[j]) : 1.f;
+        srow[j] = S + ((size_t)t.e * a.R + wr) * (a.K >> a.qsh);
+        sc_next[j] = WF == MOE_W_INT4_B32 ? __ldg(srow[j] + ((t.k0 * kBK + c8 * 8) >> a.qsh)) : 1.f;
       }
       for (int kb = 0; kb < t.nk; ++kb, ++it) {
         float sc[kPer];
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
           sc[j] = sc_next[j];
-          if (WF == MOE_W_INT4_B32 && kb + 1 < t.nk) sc_next[j] = __ldg(srow[j] + (kb + 1) * 2);
+          if (WF == MOE_W_INT4_B32 && kb + 1 < t.nk)
+            sc_next[j] = __ldg(srow[j] + (((t.k0 + kb + 1) * kBK + c8 * 8) >> a.qsh));
         }
         const int s = it % NS;
         const int ja = it % kAStages;
@@ -683,6 +687,8 @@ cudaError_t launch_gemm_gateup(const moe_desc& d, const Workspace& ws, int P, in
   a.out = ws.hbuf;
   a.R = d.I;
   a.K = d.H;
+  a.act = d.act;
+  a.qsh = d.wfmt == MOE_W_INT4_B128 ? 7 : 5;
   return launch_by_format<0>(d.wfmt, mg, mu, mb, a, num_sms, s);
 }
 
@@ -700,6 +706,7 @@ cudaError_t launch_gemm_down(const moe_desc& d, const float* topk_w, const Works
   a.out = ws.yp;
   a.R = d.H;
   a.K = d.I;
+  a.qsh = d.wfmt == MOE_W_INT4_B128 ? 7 : 5;
   return launch_by_format<1>(d.wfmt, md, md, mb, a, num_sms, s);
 }
 

@@ -94,6 +94,8 @@ struct StreamArgs {
   int stage_bytes;
   int xs_off;     // shared-memory offsets
   int ring_off;
+  int act;        // gate/up: moe_act
+  int qsh;        // int4: log2 of the scale block (5 or 7)
 };
 
 // position in the CTA's contiguous range of (touched expert, row block, token group) items
@@ -136,7 +138,7 @@ struct Cursor {
 // at xs + g*xrow + j*plane + ci*16 bytes, so a warp's reads are contiguous.
 template <int WF, int NW, int GT>
 __device__ __forceinline__ void dot_piece(const uint32_t (&rows)[NW], const float* const (&bscale)[NW],
-                                          uint32_t xs, int xrow, int plane, int k0, int nch,
+                                          uint32_t xs, int xrow, int plane, int k0, int nch, int qsh,
                                           float (&acc)[NW][kG]) {
   constexpr int V = Fmt<WF>::kVec;
   for (int c = threadIdx.x & 31; c < nch; c += 32) {
@@ -172,7 +174,7 @@ __device__ __forceinline__ void dot_piece(const uint32_t (&rows)[NW], const floa
       for (int q = 0; q < NW; ++q) {
         float wf[V];
         decode<WF>(wv[q], wf);
-        const float s = __ldg(bscale[q] + (kel >> 5));
+        const float s = __ldg(bscale[q] + (kel >> qsh));
 #pragma unroll
         for (int g = 0; g < GT; ++g) {
           float part = 0.f;
@@ -306,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const StreamAr
     for (int q = 0; q < NW; ++q) {
       const int mtx = q / RPW, rr = q % RPW;
       const float* S = mtx ? a.s1 : a.s0;
-      bsc[q] = (WF == MOE_W_INT4_B32) ? S + ((size_t)cur.e * a.R + row0 + rr) * (a.K / 32) : nullptr;
+      bsc[q] = (WF == MOE_W_INT4_B32) ? S + ((size_t)cur.e * a.R + row0 + rr) * (a.K >> a.qsh) : nullptr;
     }
     for (int p = 0; p < a.npieces; ++p, ++it) {
       const int s = it % a.NS;
@@ -326,11 +328,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const StreamAr
       const uint32_t xsa = smem_u32(xs);
       const int xrow = a.K * 4, plane = (a.K / Fmt<WF>::kVec) * 16;
       if (G == 1)
-        dot_piece<WF, NW, 1>(rows, bsc, xsa, xrow, plane, k0, nch, acc);
+        dot_piece<WF, NW, 1>(rows, bsc, xsa, xrow, plane, k0, nch, a.qsh, acc);
       else if (G == 2)
-        dot_piece<WF, NW, 2>(rows, bsc, xsa, xrow, plane, k0, nch, acc);
+        dot_piece<WF, NW, 2>(rows, bsc, xsa, xrow, plane, k0, nch, a.qsh, acc);
       else
-        dot_piece<WF, NW, kG>(rows, bsc, xsa, xrow, plane, k0, nch, acc);
+        dot_piece<WF, NW, kG>(rows, bsc, xsa, xrow, plane, k0, nch, a.qsh, acc);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
     }
@@ -357,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const StreamAr
                     gv *= a.s0[(size_t)cur.e * a.R + row];
                     uv *= a.s1[(size_t)cur.e * a.R + row];
                   }
-                  v = silu_mul(gv, uv);
+                  v = a.act == MOE_ACT_GELU_TANH ? gelu_tanh_mul(gv, uv) : silu_mul(gv, uv);
                 } else {
                   v = acc[q][gg];
                   if (WF == MOE_W_INT8_ROW) v *= a.s0[(size_t)cur.e * a.R + row];
@@ -414,8 +416,10 @@ cudaError_t launch_mode(const moe_desc& d, const StreamArgs& a, bool in_bf16, bo
   }
 }
 
-StreamArgs common_args(const Workspace& ws, int k, uint32_t* flags) {
+StreamArgs common_args(const moe_desc& d, const Workspace& ws, int k, uint32_t* flags) {
   StreamArgs a{};
+  a.act = d.act;
+  a.qsh = d.wfmt == MOE_W_INT4_B128 ? 7 : 5;
   a.offsets = ws.offsets;
   a.touched = ws.touched;
   a.group_base = ws.group_base;
@@ -433,7 +437,7 @@ static bool h_is_f32(const moe_desc& d) { return d.wfmt == MOE_W_F32; }
 
 cudaError_t launch_gemv_gateup(const moe_desc& d, const void* x, int k, const Workspace& ws, int num_sms,
                                uint32_t* flags, cudaStream_t s) {
-  StreamArgs a = common_args(ws, k, flags);
+  StreamArgs a = common_args(d, ws, k, flags);
   a.in = x;
   a.W0 = d.W_gate;
   a.W1 = d.W_up;
@@ -447,7 +451,7 @@ cudaError_t launch_gemv_gateup(const moe_desc& d, const void* x, int k, const Wo
 
 cudaError_t launch_gemv_down(const moe_desc& d, const float* topk_w, int k, const Workspace& ws, int num_sms,
                              uint32_t* flags, cudaStream_t s) {
-  StreamArgs a = common_args(ws, k, flags);
+  StreamArgs a = common_args(d, ws, k, flags);
   a.in = ws.hbuf;
   a.W0 = d.W_down;
   a.s0 = d.s_down;

@@ -103,6 +103,8 @@ cudaError_t launch_gemm_gateup(const moe_desc& d, const Workspace& ws, int P, in
                                uint32_t* flags, cudaStream_t s);
 cudaError_t launch_gemm_down(const moe_desc& d, const float* topk_w, const Workspace& ws, int P, int chunk,
                              int num_sms, uint32_t* flags, cudaStream_t s);
+cudaError_t launch_expert_counts(const int32_t* idx, int64_t n, int E, uint64_t* counts, int num_sms,
+                                 cudaStream_t s);
 cudaError_t launch_combine(const moe_desc& d, const int32_t* idx, int T, const float* yp, void* y,
                            cudaStream_t s);
 

@@ -8,6 +8,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <string>
@@ -143,12 +144,11 @@ static moe_status validate_desc(const moe_desc* d) {
   if (d->k > 32 || d->k > d->E) return fail(MOE_ERR_INVALID_ARG, "k must be <= min(E, 32) (got k=%d, E=%d)", d->k, d->E);
   if (d->router != MOE_ROUTER_SIGMOID_BIAS && d->router != MOE_ROUTER_SOFTMAX)
     return fail(MOE_ERR_INVALID_ARG, "unknown router kind %d", d->router);
-  if (d->act != MOE_ACT_SILU) {
-    if (d->act == MOE_ACT_GELU_TANH)
-      return fail(MOE_ERR_UNSUPPORTED, "unsupported activation 'gelu_tanh': this library builds SiLU only");
+  if (d->act != MOE_ACT_SILU && d->act != MOE_ACT_GELU_TANH)
     return fail(MOE_ERR_INVALID_ARG, "unknown activation %d", d->act);
-  }
-  if (d->wfmt < MOE_W_F32 || d->wfmt > MOE_W_INT4_B32) return fail(MOE_ERR_INVALID_ARG, "unknown weight format %d", d->wfmt);
+  if (d->wfmt < MOE_W_F32 || d->wfmt > MOE_W_INT4_B128) return fail(MOE_ERR_INVALID_ARG, "unknown weight format %d", d->wfmt);
+  if (d->wfmt == MOE_W_INT4_B128 && (d->H % 128 || d->I % 128))
+    return fail(MOE_ERR_INVALID_ARG, "int4 block-128 weights need H and I multiples of 128 (got %d, %d)", d->H, d->I);
   if (d->xfmt != MOE_X_F32 && d->xfmt != MOE_X_BF16) return fail(MOE_ERR_INVALID_ARG, "unknown activation dtype %d", d->xfmt);
   if (d->path < MOE_PATH_AUTO || d->path > MOE_PATH_GEMM) return fail(MOE_ERR_INVALID_ARG, "unknown path %d", d->path);
   if (!isfinite(d->scale)) return fail(MOE_ERR_INVALID_ARG, "scale must be finite");
@@ -157,7 +157,7 @@ static moe_status validate_desc(const moe_desc* d) {
     return fail(MOE_ERR_INVALID_ARG, "W_gate, W_up and W_down must be non-NULL");
   if (!aligned(d->W_gate, 16) || !aligned(d->W_up, 16) || !aligned(d->W_down, 16))
     return fail(MOE_ERR_INVALID_ARG, "expert weights must be 16-byte aligned");
-  const bool scaled = d->wfmt == MOE_W_INT8_ROW || d->wfmt == MOE_W_INT4_B32;
+  const bool scaled = d->wfmt != MOE_W_F32 && d->wfmt != MOE_W_BF16;
   if (scaled && (!d->s_gate || !d->s_up || !d->s_down))
     return fail(MOE_ERR_INVALID_ARG, "int8/int4 weights need s_gate, s_up and s_down");
   if (scaled && (!aligned(d->s_gate, 4) || !aligned(d->s_up, 4) || !aligned(d->s_down, 4)))
@@ -329,6 +329,51 @@ extern "C" moe_status moe_forward(const moe_desc* d, const void* x, int32_t T, c
     MOE_LAUNCH("gemv_down", stream, launch_gemv_down(*d, topk_w, d->k, ws, dev->num_sms, dev->flags, stream));
   }
   MOE_LAUNCH("combine", stream, launch_combine(*d, topk_idx, T, ws.yp, y, stream));
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------------ routing statistics
+
+extern "C" moe_status moe_expert_counts(const moe_desc* d, const int32_t* topk_idx, int32_t T, uint64_t* counts,
+                                        cudaStream_t stream) {
+  g_err.clear();
+  if (!d) return fail(MOE_ERR_INVALID_ARG, "descriptor is NULL");
+  if (d->E < 1 || d->E > 1024) return fail(MOE_ERR_INVALID_ARG, "E must be in [1, 1024] (got %d)", d->E);
+  if (d->k < 1 || d->k > 32) return fail(MOE_ERR_INVALID_ARG, "k must be in [1, 32] (got %d)", d->k);
+  moe_status st = validate_T(T, d->k);
+  if (st != MOE_OK) return st;
+  if (!counts || !aligned(counts, 8)) return fail(MOE_ERR_INVALID_ARG, "counts must be a non-NULL 8-byte aligned device pointer");
+  if (T == 0) return MOE_OK;
+  if (!topk_idx || !aligned(topk_idx, 4)) return fail(MOE_ERR_INVALID_ARG, "topk_idx must be non-NULL, 4-byte aligned");
+  DeviceState* dev = nullptr;
+  if ((st = device_state(&dev)) != MOE_OK) return st;
+  MOE_LAUNCH("expert_counts", stream,
+             launch_expert_counts(topk_idx, (int64_t)T * d->k, d->E, counts, dev->num_sms, stream));
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_cover_set(const uint64_t* counts, int32_t E, double cover, uint8_t* keep,
+                                    int32_t* new_index, int32_t* n_keep) {
+  g_err.clear();
+  if (!counts || !keep || !new_index || !n_keep) return fail(MOE_ERR_INVALID_ARG, "NULL argument");
+  if (E < 1) return fail(MOE_ERR_INVALID_ARG, "E must be >= 1 (got %d)", E);
+  if (!(cover > 0.0 && cover <= 1.0)) return fail(MOE_ERR_INVALID_ARG, "cover must lie in (0, 1] (got %g)", cover);
+  std::vector<int32_t> order((size_t)E);
+  uint64_t total = 0;
+  for (int32_t e = 0; e < E; ++e) {
+    order[e] = e;
+    total += counts[e];
+  }
+  std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) { return counts[a] > counts[b]; });
+  const double target = cover * (double)total;
+  int32_t m = 0;
+  uint64_t mass = 0;
+  while (m < E && (double)mass < target) mass += counts[order[m++]];
+  std::fill(keep, keep + E, (uint8_t)0);
+  for (int32_t i = 0; i < m; ++i) keep[order[i]] = 1;
+  int32_t next = 0;
+  for (int32_t e = 0; e < E; ++e) new_index[e] = keep[e] ? next++ : -1;
+  *n_keep = m;
   return MOE_OK;
 }
 

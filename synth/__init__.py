@@ -236,10 +236,11 @@ def active_mask(cfg: dict) -> Optional[np.ndarray]:
 
 
 def skew_ranks(cfg: dict, mask: np.ndarray) -> np.ndarray:
-    """Seeded rank of each active expert (0 = highest bias); -1 for masked experts."""
+    """Seeded rank of each active expert (0 = highest bias); -1 for masked experts
+    (no mask: every expert is active)."""
     E = cfg["E"]
     u = uniform_f64(E, cfg["seed"], S_RANK)
-    act = np.nonzero(mask)[0]
+    act = np.arange(E) if mask is None else np.nonzero(mask)[0]
     order = act[np.argsort(u[act], kind="stable")]
     r = np.full(E, -1, np.int64)
     r[order] = np.arange(len(order))

@@ -31,7 +31,7 @@ def layer_from_problem(prob, path=moe.MOE_PATH_AUTO) -> moe.MoELayer:
     return moe.MoELayer(H=prob.H, I=prob.I, E=prob.E, k=prob.k, router=prob.router, scale=prob.scale,
                         wfmt=prob.wfmt, xfmt=prob.xfmt, W_r=prob.W_r, b=prob.b, expert_mask=prob.mask,
                         W_gate=prob.W_gate, W_up=prob.W_up, W_down=prob.W_down, s_gate=prob.s_gate,
-                        s_up=prob.s_up, s_down=prob.s_down, path=path)
+                        s_up=prob.s_up, s_down=prob.s_down, path=path, act=prob.act)
 
 
 def x_to_device(prob) -> torch.Tensor:

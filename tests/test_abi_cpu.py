@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 import mixture_experts_layer_31_b200 as moe
@@ -52,25 +53,28 @@ def test_workspace_size_grows_with_tokens():
     ("k", 17, moe.MOE_ERR_INVALID_ARG),
     ("k", 33, moe.MOE_ERR_INVALID_ARG),
     ("E", 2048, moe.MOE_ERR_UNSUPPORTED),
-    ("act", moe.MOE_ACT_GELU_TANH, moe.MOE_ERR_UNSUPPORTED),
     ("act", 7, moe.MOE_ERR_INVALID_ARG),
     ("router", 5, moe.MOE_ERR_INVALID_ARG),
     ("wfmt", 9, moe.MOE_ERR_INVALID_ARG),
     ("W_r", None, moe.MOE_ERR_INVALID_ARG),
     ("W_gate", (1 << 20) + 4, moe.MOE_ERR_INVALID_ARG),
     ("wfmt", moe.MOE_W_INT8_ROW, moe.MOE_ERR_INVALID_ARG),  # int8 without scales
+    ("wfmt", moe.MOE_W_INT4_B128, moe.MOE_ERR_INVALID_ARG),  # block 128 needs I % 128 (I = 192 below)
 ])
 def test_invalid_descriptors_are_rejected(field, value, status):
+    extra = dict(I=192, s_gate=1 << 20, s_up=1 << 20, s_down=1 << 20) if value == moe.MOE_W_INT4_B128 else {}
     with pytest.raises(moe.MoeError) as ei:
-        moe.moe_workspace_size(_desc(**{field: value}), 16)
+        moe.moe_workspace_size(_desc(**{field: value}, **extra), 16)
     assert ei.value.status == status
     assert moe.moe_last_error()
 
 
-def test_gelu_message_names_the_activation():
-    with pytest.raises(moe.MoeError) as ei:
-        moe.moe_workspace_size(_desc(act=moe.MOE_ACT_GELU_TANH), 16)
-    assert "gelu_tanh" in str(ei.value)
+def test_both_activations_and_int4_formats_are_accepted():
+    for act in (moe.MOE_ACT_SILU, moe.MOE_ACT_GELU_TANH):
+        assert moe.moe_workspace_size(_desc(act=act), 16) > 0
+    sc = dict(s_gate=1 << 20, s_up=1 << 20, s_down=1 << 20)
+    for wfmt in (moe.MOE_W_INT4_B32, moe.MOE_W_INT4_B128):
+        assert moe.moe_workspace_size(_desc(wfmt=wfmt, **sc), 16) > 0
 
 
 def test_route_and_forward_validate_before_launch():
@@ -98,3 +102,35 @@ def test_header_declares_citations_and_ownership():
     txt = open(os.path.join(ROOT, "include", "moe.h")).read()
     for needle in ("Conversion notes", "Defrag", "owned by the caller", "MOE_ERR_UNSUPPORTED"):
         assert needle in txt
+
+
+@pytest.mark.parametrize("seed", range(5))
+@pytest.mark.parametrize("cover", [0.3, 0.95, 1.0])
+def test_cover_set_matches_oracle(seed, cover):
+    """The library's host cover-set utility against the oracle's, bit for bit
+    (host-only: no device work)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    E = int(rng.integers(1, 300))
+    counts = rng.integers(0, 50, size=E).astype(np.uint64)
+    counts[rng.random(E) < 0.3] = 0
+    counts[: E // 4] = counts[0]  # ties
+    got = moe.moe_cover_set(counts, cover)
+    ref = oracle.cover_set(counts, cover)
+    assert got[2] == ref[2]
+    np.testing.assert_array_equal(got[0], ref[0])
+    np.testing.assert_array_equal(got[1], ref[1])
+
+
+def test_cover_set_rejects_bad_arguments():
+    for cover in (0.0, -1.0, 1.01, float("nan")):
+        with pytest.raises(moe.MoeError) as ei:
+            moe.moe_cover_set(np.ones(4, np.uint64), cover)
+        assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+
+
+def test_expert_counts_validates_before_launch():
+    with pytest.raises(moe.MoeError) as ei:  # NULL counts
+        moe.moe_expert_counts(_desc(), 1 << 20, 16, None)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+    moe.moe_expert_counts(_desc(), 1 << 20, 0, 1 << 20)  # T = 0: nothing to count, nothing launched

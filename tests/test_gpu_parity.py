@@ -27,6 +27,11 @@ SMALL = {
     "kimi-int8-small": (3, dict(T=203, H=384, E=24, I=256)),
     "qwen3-int4-small": (4, dict(T=150, H=256, E=16, I=128)),
     "skew-masked-int8-small": (5, dict(T=301, H=256, E=40, I=128, n_active=23, bias=("skew", 0.15))),
+    "kimi-bf16-gelu": (2, dict(T=37, H=256, E=32, I=192, act="gelu_tanh")),
+    "kimi-int8-gelu": (3, dict(T=150, H=384, E=24, I=256, act="gelu_tanh")),
+    "tiny-fp32-gelu": (1, dict(act="gelu_tanh")),
+    "qwen3-int4b128-small": (4, dict(T=150, H=256, E=16, I=256, wfmt="int4b128")),
+    "qwen3-int4b128-gelu": (4, dict(T=77, H=384, E=12, I=128, wfmt="int4b128", act="gelu_tanh")),
 }
 
 
@@ -66,11 +71,16 @@ def test_kimi_decode_bf16_full():
     judge(prob, y, idx, w)
 
 
-@pytest.mark.parametrize("cid,n_sample", [(3, 40), (4, 96), (5, 40)])
-def test_full_workloads_sampled(cid, n_sample):
-    """Full-size prefill workloads, the same launch as the benchmark; the oracle
-    checks a seeded sample of tokens (first, last and random ones)."""
-    prob = synth.make_problem(cid)
+FULL_VARIANTS = {"int4b128": dict(wfmt="int4b128"), "gelu": dict(act="gelu_tanh")}
+
+
+@pytest.mark.parametrize("cid,n_sample,variant", [(3, 40, None), (4, 96, None), (5, 40, None),
+                                                  (4, 64, "int4b128"), (2, 32, "gelu")])
+def test_full_workloads_sampled(cid, n_sample, variant):
+    """Full-size workloads, the same launch as the benchmark (and the expert-op
+    variants at full size); the oracle checks a seeded sample of tokens (first,
+    last and random ones)."""
+    prob = synth.make_problem(cid, **FULL_VARIANTS.get(variant, {}))
     _, _, y, idx, w = run(prob)
     rng = np.random.default_rng(cid)
     toks = np.unique(np.concatenate([[0, prob.T - 1], rng.choice(prob.T, n_sample, replace=False)]))
