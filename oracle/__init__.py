@@ -72,10 +72,11 @@ def _load():
         lib.oracle_expert.argtypes = [P, i64, vp, vp]
         lib.oracle_combine.argtypes = [P, vp, i64, i64, vp, vp, vp]
         lib.oracle_forward.argtypes = [P, vp, i64, i64, vp, vp, vp, vp]
+        lib.oracle_block.argtypes = [P, P, vp, vp, i64, i64, vp, vp, vp]
         lib.oracle_expert_counts.argtypes = [vp, i64, ctypes.c_int32, vp]
         lib.oracle_cover_set.argtypes = [vp, ctypes.c_int32, ctypes.c_double, vp, vp, vp]
         for f in ("oracle_router_logits", "oracle_keys", "oracle_select", "oracle_route",
-                  "oracle_expert", "oracle_combine", "oracle_forward", "oracle_expert_counts",
+                  "oracle_expert", "oracle_combine", "oracle_forward", "oracle_block", "oracle_expert_counts",
                   "oracle_cover_set"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
@@ -106,6 +107,16 @@ class Oracle:
         L.W_gate, L.W_up, L.W_down = _p(prob.W_gate), _p(prob.W_up), _p(prob.W_down)
         L.s_gate, L.s_up, L.s_down = _p(prob.s_gate), _p(prob.s_up), _p(prob.s_down)
         self.L = L
+        self.S = None  # the shared expert as a one-expert layer, when the problem has one
+        if getattr(prob, "I_s", 0):
+            self._keep += [prob.Ws_gate, prob.Ws_up, prob.Ws_down, prob.ss_gate, prob.ss_up, prob.ss_down]
+            S = _Layer()
+            S.H, S.I, S.E, S.k = prob.H, prob.I_s, 1, 1
+            S.router, S.wfmt, S.xfmt, S.act = L.router, L.wfmt, L.xfmt, L.act
+            S.scale = 1.0
+            S.W_gate, S.W_up, S.W_down = _p(prob.Ws_gate), _p(prob.Ws_up), _p(prob.Ws_down)
+            S.s_gate, S.s_up, S.s_down = _p(prob.ss_gate), _p(prob.ss_up), _p(prob.ss_down)
+            self.S = S
         self.lib = _load()
 
     # -- helpers --------------------------------------------------------------
@@ -195,6 +206,29 @@ class Oracle:
                 i = pos[t]
                 rc = self.lib.oracle_combine(ctypes.byref(self.L), self._x(), t, t + 1,
                                              idx[i:].ctypes.data, w[i:].ctypes.data, y[i:].ctypes.data)
+                assert rc == 0
+            return 0
+
+        with ThreadPoolExecutor(self.nthreads) as ex:
+            list(ex.map(run_part, self._split(tokens)))
+        return y
+
+    def block(self, tokens: Sequence[int], idx: np.ndarray, w: np.ndarray) -> np.ndarray:
+        """The MoE block y [n,H] fp64 under a given routing: routed sum + shared expert
+        (if the problem has one) + residual (if it has one)."""
+        tokens = [int(t) for t in tokens]
+        idx = np.ascontiguousarray(idx, np.int32)
+        w = np.ascontiguousarray(w, np.float64)
+        y = np.empty((len(tokens), self.prob.H), np.float64)
+        pos = {t: i for i, t in enumerate(tokens)}
+        Sp = ctypes.byref(self.S) if self.S is not None else None
+        res = _p(getattr(self.prob, "residual", None))
+
+        def run_part(part):
+            for t in part:
+                i = pos[t]
+                rc = self.lib.oracle_block(ctypes.byref(self.L), Sp, self._x(), res, t, t + 1,
+                                           idx[i:].ctypes.data, w[i:].ctypes.data, y[i:].ctypes.data)
                 assert rc == 0
             return 0
 

@@ -304,6 +304,47 @@ int oracle_forward(const oracle_layer* L, const void* x, int64_t t0, int64_t t1,
   return rc;
 }
 
+/* ------------------------------------------------- shared expert + residual */
+/*
+ * The whole MoE block for tokens [t0, t1) under a given routing:
+ *   y[t] = sum_j w_j o_{idx_j}(x_t)  +  shared(x_t)  +  residual[t]
+ * The routed sum is oracle_combine's; shared(x) is one more gated FFN with
+ * weight 1 over every token ("256-routed + 1-shared expert FFN" -- Kimi-Linear
+ * APEX quantization page, intro; the shared expert runs beside the moe op --
+ * Kimi-Linear LiteRT-LM details page, Conversion notes, mixture-of-experts
+ * bullet), described by S as a one-expert layer (S->E == 1, same H and
+ * activation); the residual add is the block's own, outside the moe op (Qwen3
+ * card, Conversion Notes, moe_fusion_guard bullet).  S and residual may be
+ * NULL; residual is in x's format.
+ */
+int oracle_block(const oracle_layer* L, const oracle_layer* S, const void* x, const void* residual, int64_t t0,
+                 int64_t t1, const int32_t* idx, const double* w, double* y) {
+  if (S && (S->E != 1 || S->H != L->H)) return -1;
+  int rc = oracle_combine(L, x, t0, t1, idx, w, y);
+  if (rc != 0) return rc;
+  const int64_t H = L->H;
+  double* xt = (double*)malloc(sizeof(double) * H);
+  double* o = (double*)malloc(sizeof(double) * H);
+  if (!xt || !o) {
+    free(xt);
+    free(o);
+    return -1;
+  }
+  for (int64_t t = t0; t < t1 && rc == 0; ++t) {
+    double* yt = y + (t - t0) * H;
+    if (S) {
+      for (int64_t h = 0; h < H; ++h) xt[h] = x_value(L, x, t, h);
+      rc = oracle_expert(S, 0, xt, o);
+      for (int64_t h = 0; h < H; ++h) yt[h] += o[h];
+    }
+    if (residual)
+      for (int64_t h = 0; h < H; ++h) yt[h] += x_value(L, residual, t, h);
+  }
+  free(xt);
+  free(o);
+  return rc;
+}
+
 /* ------------------------------------------------------- routing statistics */
 /*
  * Per-expert routing frequencies and the covering expert set (CMF code

@@ -38,6 +38,7 @@ _lib = None
 
 # stream ids: one independent random stream per tensor
 S_X, S_WR, S_B, S_WG, S_WU, S_WD, S_MASK, S_RANK = 1, 2, 3, 4, 5, 6, 7, 8
+S_SG, S_SU, S_SD, S_RES = 9, 10, 11, 12  # shared expert gate/up/down, residual stream
 
 WFMT = {"f32": 0, "bf16": 1, "int8": 2, "int4": 3, "int4b128": 4}
 ACT = {"silu": 0, "gelu_tanh": 1}
@@ -197,6 +198,17 @@ class Problem:
     s_up: Optional[np.ndarray] = None
     s_down: Optional[np.ndarray] = None  # int8 [E,H]; int4 [E,H,I/32] (int4b128: I/128)
     act: str = "silu"                    # gated activation: "silu" or "gelu_tanh"
+    # shared expert (one dense gated FFN over every token, weight 1), stored like one
+    # routed expert ([1, I_s, H] / [1, H, I_s] and scales), and the residual stream
+    # [T, H] in x's format -- present only when the workload asks for them
+    I_s: int = 0
+    Ws_gate: Optional[np.ndarray] = None
+    Ws_up: Optional[np.ndarray] = None
+    Ws_down: Optional[np.ndarray] = None
+    ss_gate: Optional[np.ndarray] = None
+    ss_up: Optional[np.ndarray] = None
+    ss_down: Optional[np.ndarray] = None
+    residual: Optional[np.ndarray] = None
 
     def weight_bytes_per_expert(self) -> int:
         n = 0
@@ -289,7 +301,20 @@ def make_problem(cfg_id: int, nthreads: Optional[int] = None, replica: int = 0, 
     W_gate, s_gate = _expert_weights(c["wfmt"], E, I, H, seed, S_WG, g_std, nthreads)
     W_up, s_up = _expert_weights(c["wfmt"], E, I, H, seed, S_WU, g_std, nthreads)
     W_down, s_down = _expert_weights(c["wfmt"], E, H, I, seed, S_WD, d_std, nthreads)
+    extra = {}
+    I_s = int(c.get("shared") or 0)  # shared expert's intermediate size (0: none)
+    if I_s:
+        ds_std = 1.0 / math.sqrt(I_s) if c["w_std"] == "fan_in" else c["w_std"]
+        extra["I_s"] = I_s
+        extra["Ws_gate"], extra["ss_gate"] = _expert_weights(c["wfmt"], 1, I_s, H, seed, S_SG, g_std, nthreads)
+        extra["Ws_up"], extra["ss_up"] = _expert_weights(c["wfmt"], 1, I_s, H, seed, S_SU, g_std, nthreads)
+        extra["Ws_down"], extra["ss_down"] = _expert_weights(c["wfmt"], 1, H, I_s, seed, S_SD, ds_std, nthreads)
+    if c.get("residual"):
+        if c["xfmt"] == "bf16":
+            extra["residual"] = normal_bf16((T, H), x_seed, S_RES, 0.0, c["x_std"], nthreads)
+        else:
+            extra["residual"] = normal_f32((T, H), x_seed, S_RES, 0.0, c["x_std"], nthreads)
     return Problem(cfg=c, T=T, H=H, I=I, E=E, k=k, router=c["router"], scale=float(c["scale"]),
                    wfmt=c["wfmt"], xfmt=c["xfmt"], x=x, W_r=W_r, b=b, mask=mask,
                    W_gate=W_gate, W_up=W_up, W_down=W_down,
-                   s_gate=s_gate, s_up=s_up, s_down=s_down, act=c.get("act", "silu"))
+                   s_gate=s_gate, s_up=s_up, s_down=s_down, act=c.get("act", "silu"), **extra)

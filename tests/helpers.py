@@ -26,10 +26,15 @@ def problem_from_arrays(x, W_r, W_gate, W_up, W_down, k, scale, router="sigmoid"
                          s_down=f(s_down, np.float32))
 
 
-def dense_weights(prob, which):
-    """Dequantised expert matrices as float64 [E, rows, cols], decoded with numpy."""
-    W = {"gate": prob.W_gate, "up": prob.W_up, "down": prob.W_down}[which]
-    S = {"gate": prob.s_gate, "up": prob.s_up, "down": prob.s_down}[which]
+def dense_weights(prob, which, shared=False):
+    """Dequantised expert matrices as float64 [E, rows, cols] (the shared expert's as
+    [1, rows, cols] when shared), decoded with numpy."""
+    if shared:
+        W = {"gate": prob.Ws_gate, "up": prob.Ws_up, "down": prob.Ws_down}[which]
+        S = {"gate": prob.ss_gate, "up": prob.ss_up, "down": prob.ss_down}[which]
+    else:
+        W = {"gate": prob.W_gate, "up": prob.W_up, "down": prob.W_down}[which]
+        S = {"gate": prob.s_gate, "up": prob.s_up, "down": prob.s_down}[which]
     if prob.wfmt == "f32":
         return W.astype(np.float64)
     if prob.wfmt == "bf16":
@@ -49,10 +54,11 @@ def dense_weights(prob, which):
     raise ValueError(prob.wfmt)
 
 
-def dense_x(prob):
+def dense_x(prob, a=None):
+    a = prob.x if a is None else a
     if prob.xfmt == "bf16":
-        return torch.from_numpy(prob.x.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
-    return prob.x.astype(np.float64)
+        return torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+    return a.astype(np.float64)
 
 
 def textbook_swiglu(x, Wg, Wu, Wd, act="silu"):

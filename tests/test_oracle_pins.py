@@ -272,3 +272,58 @@ def test_exact_ties_break_to_lower_index(router):
     _, idx, _, _ = oracle.Oracle(prob, nthreads=1).forward()
     for t in range(prob.T):
         assert idx[t].tolist() == ([1, 3, 4] if logits[t] > 0 else [5, 1, 3])
+
+
+# ------------------------------------------------------------ shared expert + residual
+
+@pytest.mark.parametrize("act", ["silu", "gelu_tanh"])
+@pytest.mark.parametrize("wfmt,xfmt", [("f32", "f32"), ("bf16", "bf16"), ("int8", "bf16"), ("int4", "bf16")])
+def test_block_single_expert_equals_textbook(wfmt, xfmt, act):
+    """k = E = 1 with a shared expert and a residual: y = residual + scale * FFN_0(x)
+    + FFN_shared(x), against torch's activations and linear on independently decoded
+    weights (shared I differs from the routed I)."""
+    prob = synth.make_problem(1, T=4, H=64, I=64, E=1, k=1, wfmt=wfmt, xfmt=xfmt, seed=91, w_std=0.05,
+                              bias=None, act=act, shared=96, residual=True)
+    orc = oracle.Oracle(prob)
+    idx, w, _ = orc.route()
+    y = orc.block(range(prob.T), idx, w)
+    x = dense_x(prob)
+    ref = dense_x(prob, prob.residual) + prob.scale * textbook_swiglu(
+        x, dense_weights(prob, "gate")[0], dense_weights(prob, "up")[0], dense_weights(prob, "down")[0], act)
+    ref += textbook_swiglu(x, dense_weights(prob, "gate", True)[0], dense_weights(prob, "up", True)[0],
+                           dense_weights(prob, "down", True)[0], act)
+    np.testing.assert_allclose(y, ref, rtol=1e-11, atol=1e-12)
+
+
+def test_block_without_shared_or_residual_is_the_routed_sum():
+    prob = synth.make_problem(1, T=6, seed=92)
+    orc = oracle.Oracle(prob, nthreads=1)
+    idx, w, _ = orc.route()
+    np.testing.assert_array_equal(orc.block(range(6), idx, w), orc.combine(range(6), idx, w))
+
+
+def test_block_zero_shared_weights_add_only_the_residual():
+    import dataclasses
+    prob = synth.make_problem(1, T=6, seed=93, shared=64, residual=True)
+    z = dataclasses.replace(prob, Ws_gate=np.zeros_like(prob.Ws_gate))
+    orc = oracle.Oracle(z, nthreads=1)
+    idx, w, _ = orc.route()
+    np.testing.assert_array_equal(orc.block(range(6), idx, w),
+                                  orc.combine(range(6), idx, w) + prob.residual.astype(np.float64))
+
+
+def test_shared_expert_is_an_expert_with_weight_one():
+    """A shared expert with the weights of routed expert e contributes exactly
+    oracle_expert(e, x) (routing weights set to zero, no residual)."""
+    import dataclasses
+    prob = synth.make_problem(3, T=3, H=64, I=64, E=5, k=2, seed=94, shared=64)
+    e = 3
+    same = dataclasses.replace(prob, Ws_gate=prob.W_gate[e:e + 1].copy(), Ws_up=prob.W_up[e:e + 1].copy(),
+                               Ws_down=prob.W_down[e:e + 1].copy(), ss_gate=prob.s_gate[e:e + 1].copy(),
+                               ss_up=prob.s_up[e:e + 1].copy(), ss_down=prob.s_down[e:e + 1].copy())
+    orc = oracle.Oracle(same, nthreads=1)
+    idx, w, _ = orc.route()
+    y = orc.block(range(3), idx, np.zeros_like(w))
+    x = dense_x(same)
+    for t in range(3):
+        np.testing.assert_array_equal(y[t], orc.expert(e, x[t]))
