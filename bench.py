@@ -180,6 +180,12 @@ def algorithmic(prob, idx: np.ndarray):
              "gemv_down": 2.0 * P * H * I}
     layer_bytes = ut * (gate_up_per_expert + down_per_expert) + prob.W_r.nbytes + 2 * T * H * xb
     layer_flops = 6.0 * P * H * I + 2.0 * T * H * E
+    if prob.I_s:  # the block: shared expert weights (+ scales) and flops, residual read
+        layer_bytes += sum(a.nbytes for a in (prob.Ws_gate, prob.Ws_up, prob.Ws_down, prob.ss_gate, prob.ss_up,
+                                              prob.ss_down) if a is not None)
+        layer_flops += 6.0 * T * H * prob.I_s
+    if prob.residual is not None:
+        layer_bytes += T * H * xb
     return dict(touched=ut, per_expert_gate_up=gate_up_per_expert, per_expert_down=down_per_expert, bytes=bytes_,
                 flops=flops, layer_bytes=layer_bytes, layer_flops=layer_flops)
 
@@ -222,6 +228,16 @@ def cpu_threads() -> int:
         return os.cpu_count() or 1
 
 
+def oracle_step(orc, tokens):
+    """The oracle's pass over some tokens: route, experts, combine (and, for a block
+    workload, the shared expert and the residual)."""
+    p = orc.prob
+    if p.I_s or p.residual is not None:
+        idx, w, _ = orc.route(tokens)
+        return orc.block(tokens, idx, w)
+    return orc.forward(tokens)[0]
+
+
 def time_oracle(prob, budget_s: float, max_tokens=None):
     """Time the fp64 oracle (route + experts + combine) on a seeded token sample
     sized to roughly `budget_s` seconds of work; returns (tokens/s, threads, sample text)."""
@@ -229,14 +245,14 @@ def time_oracle(prob, budget_s: float, max_tokens=None):
     cores = cpu_threads()
     orc = oracle.Oracle(prob, nthreads=cores)
     t0 = time.perf_counter()
-    orc.forward([0])
+    oracle_step(orc, [0])
     per_token = max(time.perf_counter() - t0, 1e-6)  # one token, one thread
     n = int(budget_s * cores / per_token)
     n = max(1, min(n, prob.T if max_tokens is None else min(prob.T, max_tokens)))
     rng = np.random.default_rng(0)
     toks = np.sort(rng.choice(prob.T, n, replace=False))
     t0 = time.perf_counter()
-    orc.forward(toks)
+    oracle_step(orc, toks)
     dt = time.perf_counter() - t0
     return n / dt, cores, "%d of %d tokens (seeded), route + experts + combine in fp64" % (n, prob.T)
 
@@ -258,12 +274,15 @@ def run_reference(args):
     rank, world = dist_init("gloo")
     if rank != 0:
         return 0
+    if args.block:
+        args.overrides.setdefault("shared", synth.config(args.config, **args.overrides)["I"])
+        args.overrides.setdefault("residual", True)
     prob = synth.make_problem(args.config, **args.overrides)
     import oracle
     cores = cpu_threads()
     orc = oracle.Oracle(prob, nthreads=cores)
     t0 = time.perf_counter()
-    orc.forward([0])
+    oracle_step(orc, [0])
     per_token = max(time.perf_counter() - t0, 1e-6)
     # each step: a token sample worth about 6 s of oracle work on all cores
     n = max(1, min(prob.T, int(6.0 * cores / per_token)))
@@ -272,7 +291,7 @@ def run_reference(args):
     for step in range(args.warmup + args.steps):
         toks = np.sort(rng.choice(prob.T, n, replace=False))
         t0 = time.perf_counter()
-        orc.forward(toks)
+        oracle_step(orc, toks)
         dt = time.perf_counter() - t0
         if step >= args.warmup:
             times.append(dt)
@@ -281,7 +300,10 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_block(prob, args.config, {"sample_tokens_per_step": n}),
+            "config": config_block(prob, args.config, {"sample_tokens_per_step": n,
+                                                        "block": ({"shared_I": prob.I_s,
+                                                                   "residual": prob.residual is not None}
+                                                                  if args.block else None)}),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": "%d of %d tokens per step (seeded), route + experts + combine in fp64"
                                        % (n, prob.T)},
@@ -297,12 +319,17 @@ def run_ours(args):
     dist_init("nccl")
     import mixture_experts_layer_31_b200 as moe
     dev = torch.device("cuda", local)
+    if args.block:  # the whole MoE block: a shared expert of the routed size, and the residual
+        args.overrides.setdefault("shared", synth.config(args.config, **args.overrides)["I"])
+        args.overrides.setdefault("residual", True)
     prob = synth.make_problem(args.config, replica=rank, **args.overrides)
     path = {"auto": moe.MOE_PATH_AUTO, "gemv": moe.MOE_PATH_GEMV, "gemm": moe.MOE_PATH_GEMM}[args.path]
     layer = moe.MoELayer(H=prob.H, I=prob.I, E=prob.E, k=prob.k, router=prob.router, scale=prob.scale,
                          wfmt=prob.wfmt, xfmt=prob.xfmt, W_r=prob.W_r, b=prob.b, expert_mask=prob.mask,
                          W_gate=prob.W_gate, W_up=prob.W_up, W_down=prob.W_down, s_gate=prob.s_gate,
-                         s_up=prob.s_up, s_down=prob.s_down, path=path, device=dev, act=prob.act)
+                         s_up=prob.s_up, s_down=prob.s_down, path=path, device=dev, act=prob.act,
+                         I_s=prob.I_s, Ws_gate=prob.Ws_gate, Ws_up=prob.Ws_up, Ws_down=prob.Ws_down,
+                         ss_gate=prob.ss_gate, ss_up=prob.ss_up, ss_down=prob.ss_down)
     if prob.xfmt == "bf16":
         x_host = torch.from_numpy(prob.x.view(np.int16)).view(torch.bfloat16)
     else:
@@ -314,10 +341,23 @@ def run_ours(args):
     y = torch.empty((T, prob.H), dtype=layer.x_dtype, device=dev)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    counts = torch.zeros(prob.E, dtype=torch.uint64, device=dev) if args.stats else None
 
-    def step(xin, yout):
+    res_host = None
+    if prob.residual is not None:
+        res_host = torch.from_numpy(prob.residual.view(np.int16)).view(torch.bfloat16) if prob.xfmt == "bf16" \
+            else torch.from_numpy(prob.residual)
+    res = None if res_host is None else res_host.to(dev)
+
+    def step(xin, yout, rin=None):
+        rin = res if rin is None else rin
         layer.route(xin, out=(idx, w))
-        layer.forward(xin, idx, w, y=yout)
+        if counts is not None:  # routing-frequency recording (calibration runs)
+            layer.expert_counts(idx, counts)
+        if args.block:
+            layer.block(xin, idx, w, residual=rin, y=yout)
+        else:
+            layer.forward(xin, idx, w, y=yout)
 
     for _ in range(max(args.warmup, 3) if args.warmup > 0 else 0):
         step(x, y)
@@ -352,11 +392,15 @@ def run_ours(args):
     xh = x_host.pin_memory()
     yh = torch.empty(y.shape, dtype=y.dtype).pin_memory()
     xd = torch.empty_like(x)
+    rh = None if res_host is None else res_host.pin_memory()
+    rd = None if res is None else torch.empty_like(res)
     e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     for _ in range(2):
         xd.copy_(xh, non_blocking=True)
-        step(xd, y)
+        if rd is not None:
+            rd.copy_(rh, non_blocking=True)
+        step(xd, y, rd)
         yh.copy_(y, non_blocking=True)
     barrier()
     torch.cuda.synchronize(dev)
@@ -364,7 +408,9 @@ def run_ours(args):
         flush.zero_()
         e_starts[i].record(stream)
         xd.copy_(xh, non_blocking=True)
-        step(xd, y)
+        if rd is not None:
+            rd.copy_(rh, non_blocking=True)
+        step(xd, y, rd)
         yh.copy_(y, non_blocking=True)
         e_ends[i].record(stream)
     torch.cuda.synchronize(dev)
@@ -399,13 +445,18 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if prob.xfmt == "bf16" else "f32", "data": "synthetic",
             "config": config_block(prob, args.config, {"path": path_used, "touched_experts": acc["touched"],
-                                                        "overrides": args.overrides or None}),
+                                                        "overrides": args.overrides or None,
+                                                        "routing_counts": bool(args.stats),
+                                                        "block": ({"shared_I": prob.I_s,
+                                                                   "residual": prob.residual is not None}
+                                                                  if args.block else None)}),
             "roofline": roof,
             "layer": {"algorithmic_bytes": acc["layer_bytes"], "algorithmic_flops": acc["layer_flops"],
                       "hbm_frac_of_step": acc["layer_bytes"] / (step_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                       "kernels_ms": {n: round(t / max(c, 1), 5) for n, (c, t) in stages.items()}},
             "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT,
-                    "h2d_bytes_per_step": int(x.numel() * x.element_size()),
+                    "h2d_bytes_per_step": int(x.numel() * x.element_size())
+                                          + (0 if res is None else int(res.numel() * res.element_size())),
                     "d2h_bytes_per_step": int(y.numel() * y.element_size())},
             "gpu_launches": int(launches),
             "clocks": clocks.summary()}
@@ -431,6 +482,10 @@ def main(argv=None):
     ap.add_argument("--path", default="auto", choices=["auto", "gemv", "gemm"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--block", action="store_true",
+                    help="time the whole MoE block: routed experts + a shared expert of the routed size + residual")
+    ap.add_argument("--stats", action="store_true",
+                    help="also accumulate per-expert routing counts every step (moe_expert_counts)")
     ap.add_argument("--set", action="append", default=[], metavar="KEY=VAL",
                     help="override a workload field (e.g. E=64) -- for small profiling cases; not a bench line")
     args = ap.parse_args(argv)

@@ -179,6 +179,49 @@ MOE_API moe_status moe_forward_noalloc(const moe_desc* d, const void* x, int32_t
                                        const float* topk_w, void* y, cudaStream_t stream);
 
 /*
+ * The whole MoE block: routed experts + shared expert + residual.
+ *
+ *   y[t] = sum_j w[t,j] FFN_{idx[t,j]}(x[t])  +  FFN_shared(x[t])  +  residual[t]
+ *
+ * The shared expert is one more gated FFN applied to every token with weight 1
+ * ("256-routed + 1-shared expert FFN" -- Kimi-Linear APEX quantization page;
+ * the shared expert runs beside the moe op -- Kimi-Linear LiteRT-LM details
+ * page, Conversion notes).  It uses the routed experts' activation (d->act) and
+ * activation dtype; its own intermediate size I and storage format.  The
+ * residual add belongs to the block, outside the moe op (Qwen3-30B-A3B LiteRT-LM
+ * card, Conversion Notes, moe_fusion_guard bullet); it is fused here into the
+ * combine: after the k routed rows (slot order) the shared row and then the
+ * residual are added in fp32, with one rounding to y's dtype.
+ *
+ * moe_shared_expert: weights of one expert in the layouts of moe_desc with E=1:
+ *   W_gate, W_up [I, H] (int4: [I, H/2]); W_down [H, I] (int4: [H, I/2]);
+ *   scales as for one routed expert of the same format, else NULL.
+ *   I: multiple of 64 (of 128 for int4 block 128), <= 8192.
+ * moe_block_workspace_size: bytes of device workspace moe_forward_block needs
+ *   (256-byte aligned); shared may be NULL.
+ * moe_forward_block: as moe_forward, plus shared (NULL: no shared expert) and
+ *   residual ([T, H] in x's format, 16-byte aligned, or NULL: no residual).
+ *   With both NULL the result equals moe_forward's bit for bit.  y may alias
+ *   residual (each element is read before it is written, by the same thread).
+ */
+typedef struct {
+  int32_t I;
+  int32_t wfmt; /* moe_wfmt */
+  const void* W_gate;
+  const void* W_up;
+  const void* W_down;
+  const float* s_gate;
+  const float* s_up;
+  const float* s_down;
+} moe_shared_expert;
+
+MOE_API moe_status moe_block_workspace_size(const moe_desc* d, const moe_shared_expert* shared, int32_t T,
+                                            size_t* bytes);
+MOE_API moe_status moe_forward_block(const moe_desc* d, const moe_shared_expert* shared, const void* x, int32_t T,
+                                     const int32_t* topk_idx, const float* topk_w, const void* residual, void* y,
+                                     void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * Routing statistics (CMF code specialist page, How it was made: Calibrate and
  * Defrag steps).
  *

@@ -36,7 +36,8 @@ ACT = {"silu": MOE_ACT_SILU, "gelu_tanh": MOE_ACT_GELU_TANH}
 XFMT = {"f32": MOE_X_F32, "bf16": MOE_X_BF16}
 ROUTER = {"sigmoid": MOE_ROUTER_SIGMOID_BIAS, "softmax": MOE_ROUTER_SOFTMAX}
 
-EXPORTS = ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_noalloc", "moe_expert_counts",
+EXPORTS = ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_noalloc", "moe_block_workspace_size",
+           "moe_forward_block", "moe_expert_counts",
            "moe_cover_set", "moe_last_error", "moe_device_flags", "moe_launch_count", "moe_stage_timing",
            "moe_stage_times")
 MOE_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -59,6 +60,12 @@ class moe_desc(ctypes.Structure):
     ]
 
 
+class moe_shared_expert(ctypes.Structure):
+    _fields_ = [("I", ctypes.c_int32), ("wfmt", ctypes.c_int32), ("W_gate", ctypes.c_void_p),
+                ("W_up", ctypes.c_void_p), ("W_down", ctypes.c_void_p), ("s_gate", ctypes.c_void_p),
+                ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p)]
+
+
 class moe_stage_time(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int32), ("total_ms", ctypes.c_float)]
 
@@ -74,6 +81,9 @@ def _load() -> ctypes.CDLL:
     lib.moe_route.argtypes = [D, vp, i32, vp, vp, vp, sz, vp]
     lib.moe_forward.argtypes = [D, vp, i32, vp, vp, vp, vp, sz, vp]
     lib.moe_forward_noalloc.argtypes = [D, vp, i32, vp, vp, vp, vp]
+    SH = ctypes.POINTER(moe_shared_expert)
+    lib.moe_block_workspace_size.argtypes = [D, SH, i32, ctypes.POINTER(sz)]
+    lib.moe_forward_block.argtypes = [D, SH, vp, i32, vp, vp, vp, vp, vp, sz, vp]
     lib.moe_expert_counts.argtypes = [D, vp, i32, vp, vp]
     lib.moe_cover_set.argtypes = [vp, i32, ctypes.c_double, vp, vp, ctypes.POINTER(i32)]
     lib.moe_last_error.argtypes = []
@@ -83,7 +93,8 @@ def _load() -> ctypes.CDLL:
     lib.moe_launch_count.restype = ctypes.c_uint64
     lib.moe_stage_timing.argtypes = [i32]
     lib.moe_stage_times.argtypes = [ctypes.POINTER(moe_stage_time), i32, ctypes.POINTER(i32)]
-    for f in ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_noalloc", "moe_expert_counts",
+    for f in ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_noalloc", "moe_block_workspace_size",
+              "moe_forward_block", "moe_expert_counts",
               "moe_cover_set", "moe_device_flags", "moe_stage_timing", "moe_stage_times"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
@@ -128,6 +139,21 @@ def moe_forward_noalloc(desc: moe_desc, x: int, T: int, topk_idx: int, topk_w: i
     """moe_forward with the library's static scratch instead of a workspace, for
     callers that cannot allocate device memory (see include/moe.h)."""
     _check(lib().moe_forward_noalloc(ctypes.byref(desc), x, int(T), topk_idx, topk_w, y, stream))
+
+
+def moe_block_workspace_size(desc: moe_desc, shared: Optional["moe_shared_expert"], T: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().moe_block_workspace_size(ctypes.byref(desc), ctypes.byref(shared) if shared else None, int(T),
+                                          ctypes.byref(n)))
+    return n.value
+
+
+def moe_forward_block(desc: moe_desc, shared: Optional["moe_shared_expert"], x: int, T: int, topk_idx: int,
+                      topk_w: int, residual: Optional[int], y: int, workspace: int, ws_bytes: int,
+                      stream: int = 0) -> None:
+    """y = routed experts + shared expert (if any) + residual (if any)."""
+    _check(lib().moe_forward_block(ctypes.byref(desc), ctypes.byref(shared) if shared else None, x, int(T),
+                                   topk_idx, topk_w, residual, y, workspace, int(ws_bytes), stream))
 
 
 def moe_expert_counts(desc: moe_desc, topk_idx: int, T: int, counts: int, stream: int = 0) -> None:
@@ -184,7 +210,8 @@ class MoELayer:
 
     def __init__(self, *, H, I, E, k, router, scale, wfmt, xfmt, W_r, W_gate, W_up, W_down, b=None,
                  expert_mask=None, s_gate=None, s_up=None, s_down=None, path=MOE_PATH_AUTO, device="cuda",
-                 act="silu"):
+                 act="silu", I_s=0, Ws_gate=None, Ws_up=None, Ws_down=None, ss_gate=None, ss_up=None,
+                 ss_down=None):
         import torch
         lib()  # fail loudly now if the CUDA library is missing
         self.torch = torch
@@ -217,6 +244,17 @@ class MoELayer:
         self.desc = d
         self._ws = None
         self._ws_T = -1
+        self.shared = None
+        if I_s:
+            self.shared_tensors = dict(W_gate=dev(Ws_gate), W_up=dev(Ws_up), W_down=dev(Ws_down),
+                                       s_gate=dev(ss_gate), s_up=dev(ss_up), s_down=dev(ss_down))
+            sh = moe_shared_expert()
+            sh.I, sh.wfmt = int(I_s), d.wfmt
+            for name, t in self.shared_tensors.items():
+                setattr(sh, name, None if t is None else t.data_ptr())
+            self.shared = sh
+        self._bws = None
+        self._bws_T = -1
 
     @property
     def x_dtype(self):
@@ -255,6 +293,25 @@ class MoELayer:
     def __call__(self, x):
         idx, w = self.route(x)
         return self.forward(x, idx, w), idx, w
+
+    def block_workspace(self, T: int):
+        if self._bws is None or self._bws_T != T:
+            n = moe_block_workspace_size(self.desc, self.shared, T)
+            self._bws = self.torch.empty(max(n, 256), dtype=self.torch.uint8, device=self.device)
+            self._bws_T = T
+        return self._bws
+
+    def block(self, x, idx, w, residual=None, y=None):
+        """The MoE block: routed experts + the shared expert (if the layer has one) +
+        residual (if given, [T, H] in x's dtype; y may be residual itself)."""
+        T = x.shape[0]
+        if y is None:
+            y = self.torch.empty((T, self.desc.H), dtype=self.x_dtype, device=self.device)
+        ws = self.block_workspace(T)
+        moe_forward_block(self.desc, self.shared, x.data_ptr(), T, idx.data_ptr(), w.data_ptr(),
+                          None if residual is None else residual.data_ptr(), y.data_ptr(), ws.data_ptr(),
+                          ws.numel(), self._stream())
+        return y
 
     def expert_counts(self, idx, counts=None):
         """Accumulate per-expert routing counts of idx [T, k] into counts (a device

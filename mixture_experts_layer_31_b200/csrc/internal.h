@@ -106,6 +106,9 @@ cudaError_t launch_gemm_down(const moe_desc& d, const float* topk_w, const Works
 cudaError_t launch_expert_counts(const int32_t* idx, int64_t n, int E, uint64_t* counts, int num_sms,
                                  cudaStream_t s);
 cudaError_t launch_combine(const moe_desc& d, const int32_t* idx, int T, const float* yp, void* y,
-                           cudaStream_t s);
+                           cudaStream_t s, const float* ys = nullptr, const void* residual = nullptr);
+cudaError_t launch_dense_plan(int T, int chunk, int32_t* counts, int32_t* offsets, int32_t* touched,
+                              int32_t* group_base, int32_t* tile_base, int32_t* meta, int32_t* sorted_pair,
+                              float* ones, cudaStream_t s);
 
 }  // namespace moe

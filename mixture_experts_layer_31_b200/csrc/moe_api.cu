@@ -286,26 +286,10 @@ extern "C" moe_status moe_route(const moe_desc* d, const void* x, int32_t T, int
   return MOE_OK;
 }
 
-extern "C" moe_status moe_forward(const moe_desc* d, const void* x, int32_t T, const int32_t* topk_idx,
-                                  const float* topk_w, void* y, void* workspace, size_t ws_bytes,
-                                  cudaStream_t stream) {
-  g_err.clear();
-  moe_status st = validate_desc(d);
-  if (st != MOE_OK) return st;
-  if ((st = validate_T(T, d->k)) != MOE_OK) return st;
-  if (T == 0) return MOE_OK;
-  if (!x || !aligned(x, 16)) return fail(MOE_ERR_INVALID_ARG, "x must be a non-NULL 16-byte aligned device pointer");
-  if (!y || !aligned(y, 16)) return fail(MOE_ERR_INVALID_ARG, "y must be a non-NULL 16-byte aligned device pointer");
-  if (!topk_idx || !topk_w || !aligned(topk_idx, 4) || !aligned(topk_w, 4))
-    return fail(MOE_ERR_INVALID_ARG, "topk_idx and topk_w must be non-NULL, 4-byte aligned");
-  if ((st = check_ws(*d, T, workspace, ws_bytes)) != MOE_OK) return st;
-  const int path = choose_path(*d, T);
-  if (path == MOE_PATH_GEMM && !gemm_capable(*d))
-    return fail(MOE_ERR_UNSUPPORTED,
-                "tensor-core path needs bf16 activations, bf16/int8/int4 weights and H, I multiples of 128");
-  DeviceState* dev = nullptr;
-  if ((st = device_state(&dev)) != MOE_OK) return st;
-  const Workspace ws = carve_workspace(*d, T, workspace);
+// the routed experts: expert-sorted order, gate/up, down; leaves w * FFN rows in ws.yp
+static moe_status run_routed(const moe_desc* d, const void* x, int32_t T, const int32_t* topk_idx,
+                             const float* topk_w, const Workspace& ws, int path, DeviceState* dev,
+                             cudaStream_t stream) {
   const int P = T * d->k;
   const int NC = (P + kPairChunk - 1) / kPairChunk;
   if (small_sort_ok(P, d->E)) {
@@ -328,7 +312,147 @@ extern "C" moe_status moe_forward(const moe_desc* d, const void* x, int32_t T, c
     MOE_LAUNCH("gemv_gateup", stream, launch_gemv_gateup(*d, x, d->k, ws, dev->num_sms, dev->flags, stream));
     MOE_LAUNCH("gemv_down", stream, launch_gemv_down(*d, topk_w, d->k, ws, dev->num_sms, dev->flags, stream));
   }
+  return MOE_OK;
+}
+
+static moe_status check_io(const void* x, const void* y, const int32_t* topk_idx, const float* topk_w) {
+  if (!x || !aligned(x, 16)) return fail(MOE_ERR_INVALID_ARG, "x must be a non-NULL 16-byte aligned device pointer");
+  if (!y || !aligned(y, 16)) return fail(MOE_ERR_INVALID_ARG, "y must be a non-NULL 16-byte aligned device pointer");
+  if (!topk_idx || !topk_w || !aligned(topk_idx, 4) || !aligned(topk_w, 4))
+    return fail(MOE_ERR_INVALID_ARG, "topk_idx and topk_w must be non-NULL, 4-byte aligned");
+  return MOE_OK;
+}
+
+static const char* kNoTensorCores =
+    "tensor-core path needs bf16 activations, bf16/int8/int4 weights and H, I multiples of 128";
+
+extern "C" moe_status moe_forward(const moe_desc* d, const void* x, int32_t T, const int32_t* topk_idx,
+                                  const float* topk_w, void* y, void* workspace, size_t ws_bytes,
+                                  cudaStream_t stream) {
+  g_err.clear();
+  moe_status st = validate_desc(d);
+  if (st != MOE_OK) return st;
+  if ((st = validate_T(T, d->k)) != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if ((st = check_io(x, y, topk_idx, topk_w)) != MOE_OK) return st;
+  if ((st = check_ws(*d, T, workspace, ws_bytes)) != MOE_OK) return st;
+  const int path = choose_path(*d, T);
+  if (path == MOE_PATH_GEMM && !gemm_capable(*d)) return fail(MOE_ERR_UNSUPPORTED, "%s", kNoTensorCores);
+  DeviceState* dev = nullptr;
+  if ((st = device_state(&dev)) != MOE_OK) return st;
+  const Workspace ws = carve_workspace(*d, T, workspace);
+  if ((st = run_routed(d, x, T, topk_idx, topk_w, ws, path, dev, stream)) != MOE_OK) return st;
   MOE_LAUNCH("combine", stream, launch_combine(*d, topk_idx, T, ws.yp, y, stream));
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------------ the block: shared expert + residual
+
+// the shared expert as a one-expert layer: every token routed to expert 0 with weight 1
+static moe_desc shared_as_layer(const moe_desc& d, const moe_shared_expert& sh) {
+  moe_desc s = d;
+  s.E = 1;
+  s.k = 1;
+  s.I = sh.I;
+  s.wfmt = sh.wfmt;
+  s.b = nullptr;
+  s.expert_mask = nullptr;
+  s.W_gate = sh.W_gate;
+  s.W_up = sh.W_up;
+  s.W_down = sh.W_down;
+  s.s_gate = sh.s_gate;
+  s.s_up = sh.s_up;
+  s.s_down = sh.s_down;
+  return s;
+}
+
+static moe_status validate_shared(const moe_desc& d, const moe_shared_expert* sh) {
+  if (!sh) return MOE_OK;
+  if (sh->I < 64 || sh->I % 64) return fail(MOE_ERR_INVALID_ARG, "shared expert I must be a positive multiple of 64 (got %d)", sh->I);
+  if (sh->I > 8192) return fail(MOE_ERR_UNSUPPORTED, "shared expert I is limited to 8192 (got %d)", sh->I);
+  const moe_desc s = shared_as_layer(d, *sh);
+  moe_status st = validate_desc(&s);
+  if (st != MOE_OK) return fail(st, "shared expert: %s", g_err.c_str());
+  return MOE_OK;
+}
+
+// block workspace: the routed layer's, then the shared expert's (as a one-expert
+// layer over T tokens), then T unit weights
+static void block_layout(const moe_desc& d, const moe_shared_expert* sh, int32_t T, size_t* shared_off,
+                         size_t* ones_off, size_t* total) {
+  size_t off[kRegions], routed = 0, shared = 0;
+  layout(d, T, off, &routed);
+  if (sh) {
+    const moe_desc s = shared_as_layer(d, *sh);
+    layout(s, T, off, &shared);
+  }
+  *shared_off = routed;
+  *ones_off = routed + shared;
+  *total = routed + shared + (sh ? up256((size_t)T * 4) : 0);
+}
+
+extern "C" moe_status moe_block_workspace_size(const moe_desc* d, const moe_shared_expert* shared, int32_t T,
+                                               size_t* bytes) {
+  g_err.clear();
+  moe_status st = validate_desc(d);
+  if (st != MOE_OK) return st;
+  if ((st = validate_T(T, d->k)) != MOE_OK) return st;
+  if ((st = validate_shared(*d, shared)) != MOE_OK) return st;
+  if (!bytes) return fail(MOE_ERR_INVALID_ARG, "bytes is NULL");
+  size_t so, oo;
+  block_layout(*d, shared, T, &so, &oo, bytes);
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_forward_block(const moe_desc* d, const moe_shared_expert* shared, const void* x,
+                                        int32_t T, const int32_t* topk_idx, const float* topk_w,
+                                        const void* residual, void* y, void* workspace, size_t ws_bytes,
+                                        cudaStream_t stream) {
+  g_err.clear();
+  moe_status st = validate_desc(d);
+  if (st != MOE_OK) return st;
+  if ((st = validate_T(T, d->k)) != MOE_OK) return st;
+  if ((st = validate_shared(*d, shared)) != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if ((st = check_io(x, y, topk_idx, topk_w)) != MOE_OK) return st;
+  if (residual && !aligned(residual, 16)) return fail(MOE_ERR_INVALID_ARG, "residual must be 16-byte aligned");
+  size_t shared_off, ones_off, need;
+  block_layout(*d, shared, T, &shared_off, &ones_off, &need);
+  if (!workspace) return fail(MOE_ERR_WORKSPACE, "workspace is NULL (need %zu bytes)", need);
+  if (!aligned(workspace, 256)) return fail(MOE_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (ws_bytes < need) return fail(MOE_ERR_WORKSPACE, "workspace too small: %zu bytes given, %zu needed", ws_bytes, need);
+  const int path = choose_path(*d, T);
+  if (path == MOE_PATH_GEMM && !gemm_capable(*d)) return fail(MOE_ERR_UNSUPPORTED, "%s", kNoTensorCores);
+  moe_desc sd{};
+  int spath = MOE_PATH_GEMV;
+  if (shared) {
+    sd = shared_as_layer(*d, *shared);
+    spath = choose_path(sd, T);
+    if (spath == MOE_PATH_GEMM && !gemm_capable(sd)) return fail(MOE_ERR_UNSUPPORTED, "shared expert: %s", kNoTensorCores);
+  }
+  DeviceState* dev = nullptr;
+  if ((st = device_state(&dev)) != MOE_OK) return st;
+  const Workspace ws = carve_workspace(*d, T, workspace);
+  if ((st = run_routed(d, x, T, topk_idx, topk_w, ws, path, dev, stream)) != MOE_OK) return st;
+  const float* ys = nullptr;
+  if (shared) {
+    Workspace ss = carve_workspace(sd, T, static_cast<char*>(workspace) + shared_off);
+    float* ones = reinterpret_cast<float*>(static_cast<char*>(workspace) + ones_off);
+    const int chunk = chunk_tokens(T, 1, 1);
+    MOE_LAUNCH("shared_plan", stream,
+               launch_dense_plan(T, chunk, ss.counts, ss.offsets, ss.touched, ss.group_base, ss.tile_base, ss.meta,
+                                 ss.sorted_pair, ones, stream));
+    if (spath == MOE_PATH_GEMM) {
+      ss.xs = const_cast<void*>(x);  // token order is the sorted order: x serves as the gathered rows
+      MOE_LAUNCH("shared_gateup", stream, launch_gemm_gateup(sd, ss, T, chunk, dev->num_sms, dev->flags, stream));
+      MOE_LAUNCH("shared_down", stream, launch_gemm_down(sd, ones, ss, T, chunk, dev->num_sms, dev->flags, stream));
+    } else {
+      MOE_LAUNCH("shared_gateup", stream, launch_gemv_gateup(sd, x, 1, ss, dev->num_sms, dev->flags, stream));
+      MOE_LAUNCH("shared_down", stream, launch_gemv_down(sd, ones, 1, ss, dev->num_sms, dev->flags, stream));
+    }
+    ys = ss.yp;
+  }
+  MOE_LAUNCH("combine", stream, launch_combine(*d, topk_idx, T, ws.yp, y, stream, ys, residual));
   return MOE_OK;
 }
 

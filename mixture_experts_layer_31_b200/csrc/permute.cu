@@ -248,6 +248,45 @@ cudaError_t launch_expert_scan(int NC, int E, int32_t* chunk_hist, int32_t* coun
                     group_base, tile_base, chunk, meta);
 }
 
+// The plan of a dense expert applied to every token (the shared expert): the
+// sort's outputs for T pairs that all go to expert 0 in token order, and unit
+// weights, written directly.
+__global__ void __launch_bounds__(256) dense_plan_kernel(int T, int chunk, int32_t* __restrict__ counts,
+                                                         int32_t* __restrict__ offsets, int32_t* __restrict__ touched,
+                                                         int32_t* __restrict__ group_base,
+                                                         int32_t* __restrict__ tile_base, int32_t* __restrict__ meta,
+                                                         int32_t* __restrict__ sorted_pair, float* __restrict__ ones) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < T; i += gridDim.x * blockDim.x) {
+    sorted_pair[i] = i;
+    ones[i] = 1.0f;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    const int groups = (T + kGemvGroup - 1) / kGemvGroup, chunks = (T + chunk - 1) / chunk;
+    counts[0] = T;
+    offsets[0] = 0;
+    offsets[1] = T;
+    touched[0] = 0;
+    group_base[0] = 0;
+    group_base[1] = groups;
+    tile_base[0] = 0;
+    tile_base[1] = chunks;
+    meta[0] = 1;
+    meta[1] = T;
+    meta[2] = groups;
+    meta[3] = chunks;
+  }
+}
+
+cudaError_t launch_dense_plan(int T, int chunk, int32_t* counts, int32_t* offsets, int32_t* touched,
+                              int32_t* group_base, int32_t* tile_base, int32_t* meta, int32_t* sorted_pair,
+                              float* ones, cudaStream_t s) {
+  int blocks = (T + 255) / 256;
+  if (blocks > 148) blocks = 148;
+  if (blocks < 1) blocks = 1;
+  return launch_k(dense_plan_kernel, dim3(blocks), dim3(256), 0, s, T, chunk, counts, offsets, touched, group_base,
+                  tile_base, meta, sorted_pair, ones);
+}
+
 cudaError_t launch_pair_scatter(const int32_t* idx, int P, int E, const int32_t* chunk_base, int32_t* sorted_pair,
                                 cudaStream_t s) {
   const int NC = (P + kPairChunk - 1) / kPairChunk;

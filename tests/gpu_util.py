@@ -31,13 +31,17 @@ def layer_from_problem(prob, path=moe.MOE_PATH_AUTO) -> moe.MoELayer:
     return moe.MoELayer(H=prob.H, I=prob.I, E=prob.E, k=prob.k, router=prob.router, scale=prob.scale,
                         wfmt=prob.wfmt, xfmt=prob.xfmt, W_r=prob.W_r, b=prob.b, expert_mask=prob.mask,
                         W_gate=prob.W_gate, W_up=prob.W_up, W_down=prob.W_down, s_gate=prob.s_gate,
-                        s_up=prob.s_up, s_down=prob.s_down, path=path, act=prob.act)
+                        s_up=prob.s_up, s_down=prob.s_down, path=path, act=prob.act, I_s=prob.I_s,
+                        Ws_gate=prob.Ws_gate, Ws_up=prob.Ws_up, Ws_down=prob.Ws_down, ss_gate=prob.ss_gate,
+                        ss_up=prob.ss_up, ss_down=prob.ss_down)
 
 
-def x_to_device(prob) -> torch.Tensor:
+def x_to_device(prob, a=None) -> torch.Tensor:
+    """x (or another [T, H] array in x's format, e.g. the residual) on the GPU."""
+    a = prob.x if a is None else a
     if prob.xfmt == "bf16":
-        return torch.from_numpy(prob.x.view(np.int16)).view(torch.bfloat16).cuda()
-    return torch.from_numpy(prob.x).cuda()
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(a).cuda()
 
 
 def run(prob, path=moe.MOE_PATH_AUTO, layer=None):
@@ -77,3 +81,18 @@ def judge(prob, y, idx, w, tokens=None, orc=None, tol=None):
     tol = tolerance(prob) if tol is None else tol
     assert rel <= tol, "relative L2 error %.3e above %.1e" % (rel, tol)
     return dict(tokens=int(tokens.size), near_ties=int(near.size), rel_l2=rel)
+
+
+def judge_block(prob, y, idx, w, tokens=None, orc=None, tol=None):
+    """Block output (routed + shared + residual) against the oracle's block under the
+    GPU's own routing, which judge() has already held to the routing rules."""
+    tokens = np.arange(prob.T) if tokens is None else np.asarray(tokens)
+    orc = orc or oracle.Oracle(prob)
+    gi = idx.cpu().numpy()[tokens]
+    gw = w.cpu().numpy()[tokens].astype(np.float64)
+    y_ref = orc.block(tokens, gi, gw)
+    yg = y.double().cpu().numpy()[tokens]
+    rel = float(np.linalg.norm(yg - y_ref) / max(np.linalg.norm(y_ref), 1e-300))
+    tol = tolerance(prob) if tol is None else tol
+    assert rel <= tol, "block: relative L2 error %.3e above %.1e" % (rel, tol)
+    return dict(tokens=int(tokens.size), rel_l2=rel)

@@ -134,3 +134,21 @@ def test_expert_counts_validates_before_launch():
         moe.moe_expert_counts(_desc(), 1 << 20, 16, None)
     assert ei.value.status == moe.MOE_ERR_INVALID_ARG
     moe.moe_expert_counts(_desc(), 1 << 20, 0, 1 << 20)  # T = 0: nothing to count, nothing launched
+
+
+def test_block_workspace_covers_the_shared_expert():
+    d = _desc()
+    sh = moe.moe_shared_expert()
+    sh.I, sh.wfmt = 256, moe.MOE_W_BF16
+    sh.W_gate = sh.W_up = sh.W_down = 1 << 20
+    plain = moe.moe_workspace_size(d, 64)
+    assert moe.moe_block_workspace_size(d, None, 64) == plain
+    assert moe.moe_block_workspace_size(d, sh, 64) > plain
+    sh.I = 96
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_block_workspace_size(d, sh, 64)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+    sh.I, sh.wfmt = 256, moe.MOE_W_INT8_ROW  # int8 without scales
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_block_workspace_size(d, sh, 64)
+    assert "shared expert" in str(ei.value)
