@@ -19,10 +19,16 @@
 // (Qwen3 card, Available Artifacts table) is widened to q*s in bf16.
 //
 // Roles in a persistent CTA (one per SM), all walking one list of units:
-//   warp 0 lane 0   TMA producer (weight or raw quantised tiles, token boxes)
+//   warp 0 lane 0   TMA producer: bf16 weight tiles and token boxes into one
+//                   stage ring; quantised weights: raw tiles into their own ring
 //   warp 1          TMEM allocator; lane 0 issues tcgen05.mma, commits stages
+//   warp 2 lane 0   quantised weights only: TMA producer of the token boxes
 //   warps 4..11     epilogue (two 4-warp groups): tcgen05.ld -> activation / scales -> global
 //   warps 12..19    dequantisation (int8 / int4 only)
+// Quantised weights keep two rings so that a raw tile's slot is refilled as
+// soon as the dequant warps have widened it, not when the MMAs that use its
+// bf16 copy finish: the weight stream runs as many stages ahead as the raw
+// ring holds, while the token ring only needs to cover L2 latency.
 // TMEM holds two accumulator buffers when they fit (chunks up to 128 tokens),
 // so the epilogue of one unit overlaps the MMAs of the next.  Every wait is
 // bounded (MOE_FLAG_TIMEOUT).
@@ -39,7 +45,7 @@ constexpr int kBM = 128;                   // MMA M (weight rows per tile)
 constexpr int kBK = 64;                    // K per stage: one 128-byte swizzle row of bf16
 constexpr int kTileBytes = kBM * kBK * 2;  // A tile, 16 KB
 constexpr int kBoxRows = 32;               // token rows per TMA box
-constexpr int kMaxStages = 8;
+constexpr int kMaxStages = 16;
 constexpr int kAStages = 2;                // quantised: bf16 A tiles between dequant and MMA
 constexpr int kBarrierBytes = 1024;
 constexpr int kSmemLimit = 232448;         // 227 KB opt-in
@@ -58,10 +64,12 @@ struct GemmArgs {
   int R;                // weight rows per expert and matrix (I for gate/up, H for down)
   int K;                // reduction length
   int chunk;            // tokens per chunk (multiple of 16, <= 256)
-  int NS;               // pipeline stages
+  int NS;               // stages of the main ring (bf16: A and B; quantised: B only)
   int stage_bytes;
   int b_off;            // B tile offset within a stage
-  int raw_off;          // raw quantised tile offset within a stage
+  int RS;               // quantised: stages of the raw weight ring
+  int raw_stage_bytes;  // quantised: bytes of one raw stage (MT raw tiles)
+  int raw_ring_off;     // quantised: raw ring offset from the main ring's start
   int acc_stride;       // TMEM columns per M tile accumulator (power of two >= chunk)
   int nbuf;             // accumulator buffers (2: epilogue overlaps the next unit's MMAs)
   int tmem_cols;        // TMEM columns allocated
@@ -124,16 +132,23 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u, int nib, i
   return t;
 }
 
+// Raw bytes of one 8-element chunk: 8 bytes of int8, or 4 bytes of packed int4
+// (in .x).
+template <int WF>
+__device__ __forceinline__ uint2 load_chunk(const uint8_t* raw_chunk) {
+  if constexpr (WF == MOE_W_INT8_ROW) return *reinterpret_cast<const uint2*>(raw_chunk);
+  return make_uint2(*reinterpret_cast<const uint32_t*>(raw_chunk), 0u);
+}
+
 // Widen one 8-element chunk of a raw quantised row to bf16.
 // int8: byte-permute (q + 128) into the low byte of the fp32 2^23 and subtract
 // 2^23 + 128 -> exact q; |q| <= 128 has <= 8 significant bits, so the top half
 // of that fp32 is the exact bf16.  int4: same for the nibble, then q * s
 // rounded to nearest even.
 template <int WF>
-__device__ __forceinline__ uint4 widen8(const uint8_t* raw_chunk, float scale) {
+__device__ __forceinline__ uint4 widen8(const uint2 w, float scale) {
   uint32_t o[4];
   if constexpr (WF == MOE_W_INT8_ROW) {
-    const uint2 w = *reinterpret_cast<const uint2*>(raw_chunk);
     const uint32_t words[2] = {w.x ^ 0x80808080u, w.y ^ 0x80808080u};
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -145,9 +160,8 @@ __device__ __forceinline__ uint4 widen8(const uint8_t* raw_chunk, float scale) {
       o[2 * h + 1] = __byte_perm(__float_as_uint(f[2]), __float_as_uint(f[3]), 0x7632);
     }
   } else {
-    const uint32_t w = *reinterpret_cast<const uint32_t*>(raw_chunk);
-    const uint32_t lo = (w & 0x0F0F0F0Fu) ^ 0x08080808u;         // even elements, q + 8
-    const uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;  // odd elements
+    const uint32_t lo = (w.x & 0x0F0F0F0Fu) ^ 0x08080808u;         // even elements, q + 8
+    const uint32_t hi = ((w.x >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;  // odd elements
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const float q0 = __uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7440u | j)) - 8388616.0f;
@@ -181,9 +195,11 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_base + 1023u) & ~1023u) - raw_base);  // 1024-aligned
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem);  // TMA landed (A or raw, and B)
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);  // TMA landed (bf16: A and B; quantised: B)
   uint64_t* empty = full + kMaxStages;                 // MMAs finished reading the stage
-  uint64_t* ready = empty + kMaxStages;                // [kAStages] quantised: bf16 A written
+  uint64_t* rfull = empty + kMaxStages;                // quantised: raw tiles landed
+  uint64_t* rempty = rfull + kMaxStages;               // quantised: dequant warps done with the raw tiles
+  uint64_t* ready = rempty + kMaxStages;               // [kAStages] quantised: bf16 A written
   uint64_t* a_empty = ready + kAStages;                // [kAStages] quantised: MMAs done with bf16 A
   uint64_t* acc_full = a_empty + kAStages;             // [2]
   uint64_t* acc_empty = acc_full + 2;                  // [2]
@@ -192,6 +208,7 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
   float* xchg = reinterpret_cast<float*>(smem + kBarrierBytes);
   uint8_t* a_ring = smem + kBarrierBytes + Tr::kXchg;  // quantised: kAStages x MT bf16 A tiles
   uint8_t* stages = a_ring + (Tr::kQuant ? kAStages * MT * kTileBytes : 0);
+  uint8_t* raw_ring = stages + a.raw_ring_off;  // quantised only
 
   const int w = warp_id(), lane = lane_id();
   const int NS = a.NS, nbuf = a.nbuf;
@@ -200,6 +217,10 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
     for (int i = 0; i < NS; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < (Tr::kQuant ? a.RS : 0); ++i) {
+      mbar_init(&rfull[i], 1);
+      mbar_init(&rempty[i], Tr::kDequantWarps > 0 ? Tr::kDequantWarps : 1);
     }
     for (int i = 0; i < kAStages; ++i) {
       mbar_init(&ready[i], Tr::kDequantWarps > 0 ? Tr::kDequantWarps : 1);
@@ -228,39 +249,52 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
   const int total = MODE == 2 ? nib * ((a.T + a.chunk - 1) / a.chunk) * a.S
                               : (ntouched > 0 ? a.meta[3] * nib : 0);
 
-  if (w == 0) {
-    // ------------------------------------------------------------------ TMA producer
+  if (w == 0 || (Tr::kQuant && w == 2)) {
+    // ------------------------------------------------------------------ TMA producers
+    // bf16: warp 0 loads A and B into one stage.  Quantised: warp 0 loads the raw
+    // tiles into the raw ring, warp 2 the token boxes into the main ring.
     if (lane == 0) {
+      const bool load_a = w == 0, load_b = !Tr::kQuant || w == 2;
+      const bool raw = Tr::kQuant && load_a;
+      const int ring = raw ? a.RS : NS;
+      uint64_t* rf = raw ? rfull : full;
+      uint64_t* re = raw ? rempty : empty;
       bool dead = false;
       uint32_t it = 0;
-      const uint32_t abytes = MT * (Tr::kQuant ? Tr::kRawTile : kTileBytes);
+      const uint32_t abytes = load_a ? MT * (Tr::kQuant ? Tr::kRawTile : kTileBytes) : 0;
       for (int u = blockIdx.x; u < total; u += gridDim.x) {
         const Unit t = decode_unit<MODE>(a, u, nib, ntouched);
-        const int nbox = (t.n_tok + kBoxRows - 1) / kBoxRows;
+        const int nbox = load_b ? (t.n_tok + kBoxRows - 1) / kBoxRows : 0;
         const int brow = MODE == 2 ? t.base : t.base + t.c * a.chunk;
         const int wrow0 = t.e * a.R + t.ib * Tr::kRows;
         for (int kb = t.k0; kb < t.k0 + t.nk; ++kb, ++it) {
-          const int s = it % NS;
-          wait_or_die(&empty[s], ((it / NS) & 1u) ^ 1u, dead, a.flags);
+          const int s = it % ring;
+          wait_or_die(&re[s], ((it / ring) & 1u) ^ 1u, dead, a.flags);
           if (dead) continue;
-          uint8_t* st = stages + (size_t)s * a.stage_bytes;
-          mbar_arrive_expect_tx(&full[s], abytes + nbox * kBoxRows * kBK * 2);
-          const int wcol = WF == MOE_W_INT4_B32 ? kb * (kBK / 2) : kb * kBK;  // int4 maps count bytes
+          mbar_arrive_expect_tx(&rf[s], abytes + nbox * kBoxRows * kBK * 2);
+          if (load_a) {
+            uint8_t* ad = raw ? raw_ring + (size_t)s * a.raw_stage_bytes : stages + (size_t)s * a.stage_bytes;
+            const int wcol = WF == MOE_W_INT4_B32 ? kb * (kBK / 2) : kb * kBK;  // int4 maps count bytes
 #pragma unroll
-          for (int mt = 0; mt < MT; ++mt) {
-            uint8_t* adst = Tr::kQuant ? st + a.raw_off + mt * Tr::kRawTile : st + mt * kTileBytes;
-            if (MODE == 0)  // tile 0: 128 gate rows, tile 1: the same 128 up rows
-              tma_load_2d(adst, mt ? &tm_w1 : &tm_w0, wcol, wrow0, &full[s]);
-            else            // 128 down rows per tile
-              tma_load_2d(adst, &tm_w0, wcol, wrow0 + mt * kBM, &full[s]);
+            for (int mt = 0; mt < MT; ++mt) {
+              uint8_t* adst = ad + mt * (Tr::kQuant ? Tr::kRawTile : kTileBytes);
+              if (MODE == 0)  // tile 0: 128 gate rows, tile 1: the same 128 up rows
+                tma_load_2d(adst, mt ? &tm_w1 : &tm_w0, wcol, wrow0, &rf[s]);
+              else            // 128 down rows per tile
+                tma_load_2d(adst, &tm_w0, wcol, wrow0 + mt * kBM, &rf[s]);
+            }
           }
-          const int bcol = MODE == 2 ? (kb * kBK) % a.Hx : kb * kBK;
-          for (int j = 0; j < nbox; ++j)
-            tma_load_2d(st + a.b_off + j * kBoxRows * kBK * 2, &tm_b, bcol, brow + kBoxRows * j, &full[s]);
+          if (load_b) {
+            uint8_t* st = stages + (size_t)s * a.stage_bytes;
+            const int bcol = MODE == 2 ? (kb * kBK) % a.Hx : kb * kBK;
+            for (int j = 0; j < nbox; ++j)
+              tma_load_2d(st + a.b_off + j * kBoxRows * kBK * 2, &tm_b, bcol, brow + kBoxRows * j, &rf[s]);
+          }
         }
       }
-      const uint32_t first = it > (uint32_t)NS ? it - NS : 0u;
-      for (uint32_t j = first; j < it && !dead; ++j) wait_or_die(&full[j % NS], (j / NS) & 1u, dead, a.flags);
+      // let the last loads land before the CTA can exit
+      const uint32_t first = it > (uint32_t)ring ? it - ring : 0u;
+      for (uint32_t j = first; j < it && !dead; ++j) wait_or_die(&rf[j % ring], (j / ring) & 1u, dead, a.flags);
     }
   } else if (w == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -432,24 +466,34 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
           if (WF == MOE_W_INT4_B32 && kb + 1 < t.nk)
             sc_next[j] = __ldg(srow[j] + (((t.k0 + kb + 1) * kBK + c8 * 8) >> a.qsh));
         }
-        const int s = it % NS;
+        const int s = it % a.RS;
         const int ja = it % kAStages;
-        wait_or_die(&full[s], (it / NS) & 1u, dead, a.flags);
+        wait_or_die(&rfull[s], (it / a.RS) & 1u, dead, a.flags);
         wait_or_die(&a_empty[ja], ((it / kAStages) & 1u) ^ 1u, dead, a.flags);
         if (!dead) {
-          const uint8_t* raw = stages + (size_t)s * a.stage_bytes + a.raw_off;
+          const uint8_t* raw = raw_ring + (size_t)s * a.raw_stage_bytes;
           uint8_t* A = a_ring + ja * (MT * kTileBytes);
+          // all loads first, then the independent widen+store chains
+          uint2 q[kPer];
 #pragma unroll
           for (int j = 0; j < kPer; ++j) {
             const int r = r0 + kRowStep * j;
             const int mt = r >> 7, rr = r & 127;
-            const uint4 v = widen8<WF>(raw + mt * Tr::kRawTile + rr * Tr::kRawPitch + c8 * (Tr::kRawPitch / 8), sc[j]);
-            *reinterpret_cast<uint4*>(A + mt * kTileBytes + rr * 128 + ((c8 ^ (rr & 7)) << 4)) = v;
+            q[j] = load_chunk<WF>(raw + mt * Tr::kRawTile + rr * Tr::kRawPitch + c8 * (Tr::kRawPitch / 8));
+          }
+#pragma unroll
+          for (int j = 0; j < kPer; ++j) {
+            const int r = r0 + kRowStep * j;
+            const int mt = r >> 7, rr = r & 127;
+            *reinterpret_cast<uint4*>(A + mt * kTileBytes + rr * 128 + ((c8 ^ (rr & 7)) << 4)) = widen8<WF>(q[j], sc[j]);
           }
           fence_proxy_async_smem();
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ready[ja]);
+        if (lane == 0) {
+          mbar_arrive(&rempty[s]);  // the raw slot may be refilled
+          mbar_arrive(&ready[ja]);
+        }
       }
     }
   }
@@ -513,20 +557,36 @@ template <int MODE, int WF, int MT>
 cudaError_t launch_gemm(const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb, GemmArgs a,
                         int num_sms, cudaStream_t s) {
   using Tr = Traits<MODE, WF, MT>;
-  // stage: bf16 weights [A: MT x 16 KB][B]; quantised [B][raw: MT tiles] (their bf16 A lives
-  // in the A ring).  Token boxes are kBoxRows tall: B holds the chunk rounded up to whole boxes.
+  // stage: bf16 weights [A: MT x 16 KB][B]; quantised [B], with the raw tiles in a ring of
+  // their own after the main ring (their bf16 A lives in the A ring).  Token boxes are
+  // kBoxRows tall: B holds the chunk rounded up to whole boxes.  All sizes are multiples of
+  // 1024 (4 KB boxes, 16/8/4 KB tiles).
   const int b_rows = (a.chunk + kBoxRows - 1) / kBoxRows * kBoxRows;
   a.b_off = Tr::kQuant ? 0 : MT * kTileBytes;
-  a.raw_off = a.b_off + b_rows * kBK * 2;
-  a.stage_bytes = a.raw_off + MT * Tr::kRawTile;  // multiple of 1024 (4 KB boxes, 16/8/4 KB tiles)
+  a.stage_bytes = a.b_off + b_rows * kBK * 2;
+  a.raw_stage_bytes = MT * Tr::kRawTile;
   a.acc_stride = (int)pow2_at_least((uint32_t)a.chunk);
   a.nbuf = 2 * MT * a.acc_stride <= 512 ? 2 : 1;
   a.tmem_cols = a.nbuf * MT * a.acc_stride;
   const int fixed = 1024 + kBarrierBytes + Tr::kXchg + (Tr::kQuant ? kAStages * MT * kTileBytes : 0);
-  a.NS = (kSmemLimit - fixed) / a.stage_bytes;
-  if (a.NS > kMaxStages) a.NS = kMaxStages;
+  const int avail = kSmemLimit - fixed;
+  if (Tr::kQuant) {
+    // token ring: about 96 KB of boxes (L2-resident rows), 2..4 stages; the rest feeds the
+    // raw weight ring (HBM latency)
+    a.NS = (96 * 1024) / a.stage_bytes;
+    a.NS = a.NS < 2 ? 2 : (a.NS > 4 ? 4 : a.NS);
+    a.RS = (avail - a.NS * a.stage_bytes) / a.raw_stage_bytes;
+    while (a.RS < 3 && a.NS > 2) a.RS = (avail - --a.NS * a.stage_bytes) / a.raw_stage_bytes;
+    if (a.RS > kMaxStages) a.RS = kMaxStages;
+    if (a.RS < 2) return cudaErrorInvalidConfiguration;
+  } else {
+    a.NS = avail / a.stage_bytes;
+    if (a.NS > kMaxStages) a.NS = kMaxStages;
+    a.RS = 0;
+  }
   if (a.NS < 2) return cudaErrorInvalidConfiguration;
-  const size_t smem = (size_t)fixed + (size_t)a.NS * a.stage_bytes;
+  a.raw_ring_off = a.NS * a.stage_bytes;
+  const size_t smem = (size_t)fixed + (size_t)a.NS * a.stage_bytes + (size_t)a.RS * a.raw_stage_bytes;
   auto kern = gemm_tc_kernel<MODE, WF, MT>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
