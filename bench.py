@@ -4,7 +4,8 @@
 
 One step = one pass of the whole layer (router -> expert-sorted order ->
 gate/up -> down -> combine) over one batch of the workload, through the C ABI
-(moe_route + moe_forward).  Default workload: the Kimi-shaped decode batch
+(moe_layer_forward; with --block or --stats: moe_route, then
+moe_forward_block or moe_expert_counts + moe_forward).  Default workload: the Kimi-shaped decode batch
 (T=32, H=2304, E=256, k=8, I=2048, bf16 weights).
 
   value  tokens/s over the timed steps, inputs resident in HBM; each step timed
@@ -351,6 +352,9 @@ def run_ours(args):
 
     def step(xin, yout, rin=None):
         rin = res if rin is None else rin
+        if not args.block and counts is None:  # the layer in one call (moe_layer_forward)
+            layer.layer(xin, out=(yout, idx, w))
+            return
         layer.route(xin, out=(idx, w))
         if counts is not None:  # routing-frequency recording (calibration runs)
             layer.expert_counts(idx, counts)

@@ -179,6 +179,18 @@ MOE_API moe_status moe_forward_noalloc(const moe_desc* d, const void* x, int32_t
                                        const float* topk_w, void* y, cudaStream_t stream);
 
 /*
+ * Route and forward in one call: the same results as moe_route followed by
+ * moe_forward on the same arguments (topk_idx and topk_w are outputs here, as
+ * for moe_route; the workspace is moe_workspace_size's).  Because the library
+ * builds the routing itself, decode-sized batches (T <= 32, E <= 256) compute
+ * the router logits in one kernel and the top-k together with the expert sort
+ * in a second one, instead of four launches.  Larger batches run the two steps
+ * as the separate entry points do.
+ */
+MOE_API moe_status moe_layer_forward(const moe_desc* d, const void* x, int32_t T, int32_t* topk_idx, float* topk_w,
+                                     void* y, void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * The whole MoE block: routed experts + shared expert + residual.
  *
  *   y[t] = sum_j w[t,j] FFN_{idx[t,j]}(x[t])  +  FFN_shared(x[t])  +  residual[t]

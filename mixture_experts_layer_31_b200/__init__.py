@@ -36,7 +36,8 @@ ACT = {"silu": MOE_ACT_SILU, "gelu_tanh": MOE_ACT_GELU_TANH}
 XFMT = {"f32": MOE_X_F32, "bf16": MOE_X_BF16}
 ROUTER = {"sigmoid": MOE_ROUTER_SIGMOID_BIAS, "softmax": MOE_ROUTER_SOFTMAX}
 
-EXPORTS = ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_noalloc", "moe_block_workspace_size",
+EXPORTS = ("moe_workspace_size", "moe_route", "moe_forward", "moe_layer_forward", "moe_forward_noalloc",
+           "moe_block_workspace_size",
            "moe_forward_block", "moe_expert_counts",
            "moe_cover_set", "moe_last_error", "moe_device_flags", "moe_launch_count", "moe_stage_timing",
            "moe_stage_times")
@@ -81,6 +82,7 @@ def _load() -> ctypes.CDLL:
     lib.moe_route.argtypes = [D, vp, i32, vp, vp, vp, sz, vp]
     lib.moe_forward.argtypes = [D, vp, i32, vp, vp, vp, vp, sz, vp]
     lib.moe_forward_noalloc.argtypes = [D, vp, i32, vp, vp, vp, vp]
+    lib.moe_layer_forward.argtypes = [D, vp, i32, vp, vp, vp, vp, sz, vp]
     SH = ctypes.POINTER(moe_shared_expert)
     lib.moe_block_workspace_size.argtypes = [D, SH, i32, ctypes.POINTER(sz)]
     lib.moe_forward_block.argtypes = [D, SH, vp, i32, vp, vp, vp, vp, vp, sz, vp]
@@ -93,7 +95,8 @@ def _load() -> ctypes.CDLL:
     lib.moe_launch_count.restype = ctypes.c_uint64
     lib.moe_stage_timing.argtypes = [i32]
     lib.moe_stage_times.argtypes = [ctypes.POINTER(moe_stage_time), i32, ctypes.POINTER(i32)]
-    for f in ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_noalloc", "moe_block_workspace_size",
+    for f in ("moe_workspace_size", "moe_route", "moe_forward", "moe_layer_forward", "moe_forward_noalloc",
+              "moe_block_workspace_size",
               "moe_forward_block", "moe_expert_counts",
               "moe_cover_set", "moe_device_flags", "moe_stage_timing", "moe_stage_times"):
         getattr(lib, f).restype = ctypes.c_int
@@ -132,6 +135,13 @@ def moe_route(desc: moe_desc, x: int, T: int, topk_idx: int, topk_w: int, worksp
 def moe_forward(desc: moe_desc, x: int, T: int, topk_idx: int, topk_w: int, y: int, workspace: int,
                 ws_bytes: int, stream: int = 0) -> None:
     _check(lib().moe_forward(ctypes.byref(desc), x, int(T), topk_idx, topk_w, y, workspace, int(ws_bytes), stream))
+
+
+def moe_layer_forward(desc: moe_desc, x: int, T: int, topk_idx: int, topk_w: int, y: int, workspace: int,
+                      ws_bytes: int, stream: int = 0) -> None:
+    """moe_route + moe_forward in one call (topk_idx / topk_w are written)."""
+    _check(lib().moe_layer_forward(ctypes.byref(desc), x, int(T), topk_idx, topk_w, y, workspace, int(ws_bytes),
+                                   stream))
 
 
 def moe_forward_noalloc(desc: moe_desc, x: int, T: int, topk_idx: int, topk_w: int, y: int,
@@ -293,6 +303,20 @@ class MoELayer:
     def __call__(self, x):
         idx, w = self.route(x)
         return self.forward(x, idx, w), idx, w
+
+    def layer(self, x, out=None):
+        """Route and forward in one call (moe_layer_forward): (y, idx, w)."""
+        T = x.shape[0]
+        if out is None:
+            idx = self.torch.empty((T, self.desc.k), dtype=self.torch.int32, device=self.device)
+            w = self.torch.empty((T, self.desc.k), dtype=self.torch.float32, device=self.device)
+            y = self.torch.empty((T, self.desc.H), dtype=self.x_dtype, device=self.device)
+        else:
+            y, idx, w = out
+        ws = self.workspace(T)
+        moe_layer_forward(self.desc, x.data_ptr(), T, idx.data_ptr(), w.data_ptr(), y.data_ptr(), ws.data_ptr(),
+                          ws.numel(), self._stream())
+        return y, idx, w
 
     def block_workspace(self, T: int):
         if self._bws is None or self._bws_T != T:

@@ -103,6 +103,15 @@ cudaError_t launch_gemm_gateup(const moe_desc& d, const Workspace& ws, int P, in
                                uint32_t* flags, cudaStream_t s);
 cudaError_t launch_gemm_down(const moe_desc& d, const float* topk_w, const Workspace& ws, int P, int chunk,
                              int num_sms, uint32_t* flags, cudaStream_t s);
+// decode-sized batches (T <= 32): fp32 logits in one launch; with E <= 256 and
+// T*k <= 8192 also top-k and the expert sort in one launch
+bool decode_route_ok(const moe_desc& d, int T);
+bool fused_route_sort_ok(const moe_desc& d, int T);
+int decode_logit_splits(const moe_desc& d, int T);  // S: partial sums per logit (1, 2, 4 or 8)
+cudaError_t launch_decode_logits(const moe_desc& d, const void* x, int T, float* partial, int S, uint32_t* flags,
+                                 cudaStream_t s);
+cudaError_t launch_topk_sort(const moe_desc& d, const float* partial, int S, int T, int32_t* idx, float* w,
+                             int chunk, const Workspace& ws, uint32_t* flags, cudaStream_t s);
 cudaError_t launch_expert_counts(const int32_t* idx, int64_t n, int E, uint64_t* counts, int num_sms,
                                  cudaStream_t s);
 cudaError_t launch_combine(const moe_desc& d, const int32_t* idx, int T, const float* yp, void* y,

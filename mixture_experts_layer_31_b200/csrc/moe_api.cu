@@ -193,7 +193,8 @@ constexpr int kRegions = 13;
 static void layout(const moe_desc& d, int32_t T, size_t off[kRegions], size_t* total) {
   const size_t P = (size_t)T * d.k, E = d.E;
   const size_t S_simt = router_splits(T), S_tc = d.xfmt == MOE_X_BF16 ? router_tc_splits(T, d.H) : 0;
-  const size_t S = S_simt > S_tc ? S_simt : S_tc;
+  size_t S = S_simt > S_tc ? S_simt : S_tc;
+  if (T <= 32 && S < 8) S = 8;  // the decode router's splits (at most 8)
   const size_t w3_bytes = d.xfmt == MOE_X_BF16 ? (size_t)d.E * 3 * d.H * 2 : 0;
   const size_t NC = (P + kPairChunk - 1) / kPairChunk;
   const size_t hbytes = d.wfmt == MOE_W_F32 ? 4 : 2;
@@ -272,7 +273,12 @@ extern "C" moe_status moe_route(const moe_desc* d, const void* x, int32_t T, int
   if ((st = device_state(&dev)) != MOE_OK) return st;
   const Workspace ws = carve_workspace(*d, T, workspace);
   int S;
-  if (router_tc_supported(*d)) {
+  if (decode_route_ok(*d, T)) {
+    // decode-sized batch: fp32 logits from fp32 W_r in one launch, every H-split
+    // summed inside it
+    S = decode_logit_splits(*d, T);
+    MOE_LAUNCH("router_decode_logits", stream, launch_decode_logits(*d, x, T, ws.logits, S, dev->flags, stream));
+  } else if (router_tc_supported(*d)) {
     // tensor cores: fp32-accurate logits from bf16 x against the exact three-way bf16 split of W_r
     S = router_tc_splits(T, d->H);
     MOE_LAUNCH("router_split3", stream, launch_router_split3(*d, ws.w3, dev->num_sms, stream));
@@ -286,13 +292,16 @@ extern "C" moe_status moe_route(const moe_desc* d, const void* x, int32_t T, int
   return MOE_OK;
 }
 
-// the routed experts: expert-sorted order, gate/up, down; leaves w * FFN rows in ws.yp
+// the routed experts: expert-sorted order (unless already built), gate/up, down;
+// leaves w * FFN rows in ws.yp
 static moe_status run_routed(const moe_desc* d, const void* x, int32_t T, const int32_t* topk_idx,
                              const float* topk_w, const Workspace& ws, int path, DeviceState* dev,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, bool sorted = false) {
   const int P = T * d->k;
   const int NC = (P + kPairChunk - 1) / kPairChunk;
-  if (small_sort_ok(P, d->E)) {
+  if (sorted) {
+    // the plan was built together with the routing
+  } else if (small_sort_ok(P, d->E)) {
     MOE_LAUNCH("small_sort", stream,
                launch_small_sort(topk_idx, P, d->E, chunk_tokens(T, d->k, d->E), ws.counts, ws.offsets, ws.touched,
                                  ws.group_base, ws.tile_base, ws.meta, ws.sorted_pair, dev->flags, stream));
@@ -342,6 +351,37 @@ extern "C" moe_status moe_forward(const moe_desc* d, const void* x, int32_t T, c
   if ((st = device_state(&dev)) != MOE_OK) return st;
   const Workspace ws = carve_workspace(*d, T, workspace);
   if ((st = run_routed(d, x, T, topk_idx, topk_w, ws, path, dev, stream)) != MOE_OK) return st;
+  MOE_LAUNCH("combine", stream, launch_combine(*d, topk_idx, T, ws.yp, y, stream));
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------------ route and forward in one call
+
+extern "C" moe_status moe_layer_forward(const moe_desc* d, const void* x, int32_t T, int32_t* topk_idx,
+                                        float* topk_w, void* y, void* workspace, size_t ws_bytes,
+                                        cudaStream_t stream) {
+  g_err.clear();
+  moe_status st = validate_desc(d);
+  if (st != MOE_OK) return st;
+  if ((st = validate_T(T, d->k)) != MOE_OK) return st;
+  if (!fused_route_sort_ok(*d, T)) {
+    // larger batches: the two steps as moe_route and moe_forward run them
+    if ((st = moe_route(d, x, T, topk_idx, topk_w, workspace, ws_bytes, stream)) != MOE_OK) return st;
+    return moe_forward(d, x, T, topk_idx, topk_w, y, workspace, ws_bytes, stream);
+  }
+  if ((st = check_io(x, y, topk_idx, topk_w)) != MOE_OK) return st;
+  if ((st = check_ws(*d, T, workspace, ws_bytes)) != MOE_OK) return st;
+  const int path = choose_path(*d, T);
+  if (path == MOE_PATH_GEMM && !gemm_capable(*d)) return fail(MOE_ERR_UNSUPPORTED, "%s", kNoTensorCores);
+  DeviceState* dev = nullptr;
+  if ((st = device_state(&dev)) != MOE_OK) return st;
+  const Workspace ws = carve_workspace(*d, T, workspace);
+  const int S = decode_logit_splits(*d, T);
+  MOE_LAUNCH("router_decode_logits", stream, launch_decode_logits(*d, x, T, ws.logits, S, dev->flags, stream));
+  MOE_LAUNCH("router_topk_sort", stream,
+             launch_topk_sort(*d, ws.logits, S, T, topk_idx, topk_w, chunk_tokens(T, d->k, d->E), ws, dev->flags,
+                              stream));
+  if ((st = run_routed(d, x, T, topk_idx, topk_w, ws, path, dev, stream, true)) != MOE_OK) return st;
   MOE_LAUNCH("combine", stream, launch_combine(*d, topk_idx, T, ws.yp, y, stream));
   return MOE_OK;
 }

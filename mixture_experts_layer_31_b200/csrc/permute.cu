@@ -8,8 +8,11 @@
 // sort by expert (ties in pair order) with no order-dependent atomics.
 #include "common.cuh"
 #include "internal.h"
+#include "route_dev.cuh"
 
 namespace moe {
+using route_dev::kSmallE;
+using route_dev::kSortWarps;
 namespace {
 
 __global__ void __launch_bounds__(256) pair_histogram_kernel(const int32_t* __restrict__ idx, int P, int E,
@@ -32,33 +35,6 @@ __global__ void __launch_bounds__(256) pair_histogram_kernel(const int32_t* __re
   for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_hist[(size_t)blockIdx.x * E + e] = hist[e];
 }
 
-// exclusive prefix sum over the block (blockDim.x <= 1024); returns the block total in *total
-__device__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
-  const int lane = lane_id(), w = warp_id(), nw = blockDim.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int n = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-    if (lane >= off) incl += n;
-  }
-  if (lane == 31) warp_sums[w] = incl;
-  __syncthreads();
-  if (w == 0) {
-    int s = lane < nw ? warp_sums[lane] : 0;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int n = __shfl_up_sync(0xFFFFFFFFu, s, off);
-      if (lane >= off) s += n;
-    }
-    if (lane < nw) warp_sums[lane] = s;  // inclusive over warps
-  }
-  __syncthreads();
-  const int before = (w > 0 ? warp_sums[w - 1] : 0) + incl - v;
-  *total = warp_sums[nw - 1];
-  __syncthreads();
-  return before;
-}
-
 // one block, one thread per expert: per-chunk bases, counts, offsets, touched list
 __global__ void __launch_bounds__(1024) expert_scan_kernel(int NC, int E, int32_t* __restrict__ chunk_hist,
                                                            int32_t* __restrict__ counts,
@@ -79,24 +55,24 @@ __global__ void __launch_bounds__(1024) expert_scan_kernel(int NC, int E, int32_
     counts[e] = running;
   }
   int total;
-  const int off = block_exclusive_scan(e < E ? running : 0, warp_sums, &total);
+  const int off = route_dev::block_exclusive_scan(e < E ? running : 0, warp_sums, &total);
   if (e < E) {
     offsets[e] = off;
     for (int c = 0; c < NC; ++c) chunk_hist[(size_t)c * E + e] += off;
   }
   if (e == 0) offsets[E] = total;
   int ntouched;
-  const int tpos = block_exclusive_scan((e < E && running > 0) ? 1 : 0, warp_sums, &ntouched);
+  const int tpos = route_dev::block_exclusive_scan((e < E && running > 0) ? 1 : 0, warp_sums, &ntouched);
   if (e < E && running > 0) touched[tpos] = e;
   // token groups per touched expert, prefixed in touched (= ascending expert) order
   const int groups = (e < E) ? (running + kGemvGroup - 1) / kGemvGroup : 0;
   int ngroups;
-  const int gpos = block_exclusive_scan(groups, warp_sums, &ngroups);
+  const int gpos = route_dev::block_exclusive_scan(groups, warp_sums, &ngroups);
   if (e < E && running > 0) group_base[tpos] = gpos;
   // token chunks of the tensor-core path, same order
   const int chunks = (e < E) ? (running + chunk - 1) / chunk : 0;
   int nchunks;
-  const int cpos = block_exclusive_scan(chunks, warp_sums, &nchunks);
+  const int cpos = route_dev::block_exclusive_scan(chunks, warp_sums, &nchunks);
   if (e < E && running > 0) tile_base[tpos] = cpos;
   if (e == 0) {
     meta[0] = ntouched;
@@ -138,14 +114,6 @@ __global__ void __launch_bounds__(128) pair_scatter_kernel(const int32_t* __rest
   }
 }
 
-// Small batches: the whole sort in one CTA of 32 warps.  Warp w owns the
-// contiguous pair segment [w*seg, (w+1)*seg): it counts its pairs per expert
-// (no atomics: match_any groups equal experts, the last peer adds), the block
-// turns (warp, expert) counts into exclusive bases, and each warp re-walks its
-// segment in order to scatter.  Same stable order as the chunked kernels.
-constexpr int kSmallE = 256;
-constexpr int kSortWarps = 32;
-
 __global__ void __launch_bounds__(1024) small_sort_kernel(const int32_t* __restrict__ idx, int P, int E,
                                                           int chunk, int32_t* __restrict__ counts,
                                                           int32_t* __restrict__ offsets,
@@ -156,71 +124,8 @@ __global__ void __launch_bounds__(1024) small_sort_kernel(const int32_t* __restr
                                                           int32_t* __restrict__ sorted_pair, uint32_t* flags) {
   __shared__ int32_t base[kSortWarps][kSmallE];
   __shared__ int warp_sums[32];
-  const int w = warp_id(), lane = lane_id();
-  for (int i = threadIdx.x; i < kSortWarps * kSmallE; i += blockDim.x) (&base[0][0])[i] = 0;
-  __syncthreads();
-  const int seg = (P + kSortWarps - 1) / kSortWarps;
-  const int p0 = min(P, w * seg), p1 = min(P, p0 + seg);
-  const unsigned lt = (1u << lane) - 1u;
-  bool bad = false;
-  for (int pb = p0; pb < p1; pb += 32) {
-    const int p = pb + lane;
-    int e = (p < p1) ? idx[p] : -1;
-    if (p < p1 && (e < 0 || e >= E)) bad = true;
-    if (e < 0 || e >= E) e = -1;
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
-    if (e >= 0 && lane == 31 - __clz(peers)) base[w][e] += __popc(peers);
-  }
-  if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) raise_flag(flags, MOE_FLAG_BAD_EXPERT_INDEX);
-  __syncthreads();
-  // per expert: exclusive prefix over warps, then over experts
-  const int e = threadIdx.x;
-  int running = 0;
-  if (e < E) {
-    for (int ww = 0; ww < kSortWarps; ++ww) {
-      const int v = base[ww][e];
-      base[ww][e] = running;
-      running += v;
-    }
-    counts[e] = running;
-  }
-  int total;
-  const int off = block_exclusive_scan(e < E ? running : 0, warp_sums, &total);
-  if (e < E) {
-    offsets[e] = off;
-    for (int ww = 0; ww < kSortWarps; ++ww) base[ww][e] += off;
-  }
-  if (e == 0) offsets[E] = total;
-  int ntouched;
-  const int tpos = block_exclusive_scan((e < E && running > 0) ? 1 : 0, warp_sums, &ntouched);
-  if (e < E && running > 0) touched[tpos] = e;
-  const int groups = (e < E) ? (running + kGemvGroup - 1) / kGemvGroup : 0;
-  int ngroups;
-  const int gpos = block_exclusive_scan(groups, warp_sums, &ngroups);
-  if (e < E && running > 0) group_base[tpos] = gpos;
-  const int chunks = (e < E) ? (running + chunk - 1) / chunk : 0;
-  int nchunks;
-  const int cpos = block_exclusive_scan(chunks, warp_sums, &nchunks);
-  if (e < E && running > 0) tile_base[tpos] = cpos;
-  if (e == 0) {
-    meta[0] = ntouched;
-    meta[1] = total;
-    meta[2] = ngroups;
-    meta[3] = nchunks;
-    group_base[ntouched] = ngroups;
-    tile_base[ntouched] = nchunks;
-  }
-  __syncthreads();
-  for (int pb = p0; pb < p1; pb += 32) {
-    const int p = pb + lane;
-    int ee = (p < p1) ? idx[p] : -1;
-    if (ee < 0 || ee >= E) ee = -1;
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, ee);
-    if (ee >= 0) sorted_pair[base[w][ee] + __popc(peers & lt)] = p;
-    __syncwarp();
-    if (ee >= 0 && lane == 31 - __clz(peers)) base[w][ee] += __popc(peers);
-    __syncwarp();
-  }
+  route_dev::block_small_sort(idx, P, E, chunk, counts, offsets, touched, group_base, tile_base, meta, sorted_pair,
+                              flags, base, warp_sums);
 }
 
 }  // namespace

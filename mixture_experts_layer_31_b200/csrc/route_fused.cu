@@ -1,0 +1,209 @@
+// Router and expert sort for decode-sized batches, fused to two launches.
+//
+// "the router in plain ops (sigmoid scores, the top 8 chosen on the scores plus
+// the correction bias, weights renormalized and scaled by 2.446)" (Kimi-Linear
+// LiteRT-LM details page, Conversion notes); the sort groups the (token, slot)
+// pairs by expert so that each expert's weights stream once ("only the 8
+// routed experts are computed for each token" -- Qwen3-30B-A3B LiteRT-LM card,
+// Conversion Notes).
+//
+//   decode_logits_kernel  fp32 partial logits [S, T, E] straight from fp32
+//                         W_r (S from 1 to 8: about 128 CTAs, and a slice of
+//                         x and W_r that fits in shared memory): a CTA owns one S-th of H for
+//                         8 experts, stages that slice in shared memory (all
+//                         loads in flight at once), and its 8 warps split the
+//                         slice's K range, each lane holding a 2-expert x
+//                         4-token register tile; warps are added in a fixed
+//                         order, and the top-k adds the S slices in a fixed
+//                         order.  Every sum's order depends on H (and T) only,
+//                         so a masked layer and its sliced twin get the same
+//                         logits bit for bit.  T <= 32.
+//   topk_sort_kernel      one CTA: top-k of every token (one warp per token),
+//                         then the stable counting sort by expert of all T*k
+//                         pairs -- the same device code as the standalone
+//                         kernels, without the launch in between.
+#include "common.cuh"
+#include "internal.h"
+#include "route_dev.cuh"
+
+namespace moe {
+namespace {
+
+// decode logits: CTA (slice sl of S along H, group of kGroupE experts); the
+// slice of x (bf16 or fp32 as given, T rows) and of W_r (fp32, kGroupE rows)
+// is bulk-copied into shared memory; 8 warps split the slice's K range, every
+// lane owns a 2-expert x 4-token register tile (rows of experts past E hold
+// stale shared memory: their sums are never stored).  S (1..8) spreads the
+// work over about 128 CTAs and keeps the slice within shared memory.
+constexpr int kGroupE = 8;       // experts per CTA
+constexpr int kMaxDecodeT = 32;  // tokens
+constexpr int kLogitWarps = 8;
+constexpr int kLogitThreads = 32 * kLogitWarps;
+constexpr int kRedFloats = kLogitWarps * kGroupE * kMaxDecodeT;
+constexpr size_t kLogitSmemCap = 232448 - 64;  // 227 KB opt-in, less the static barrier
+
+template <bool XBF16>
+__host__ __device__ constexpr int x_elem_bytes() { return XBF16 ? 2 : 4; }
+
+template <bool XBF16>
+__global__ void __launch_bounds__(kLogitThreads) decode_logits_kernel(const void* __restrict__ x,
+                                                                      const float* __restrict__ Wr, int T, int H,
+                                                                      int E, int S, float* __restrict__ partial,
+                                                                      uint32_t* flags) {
+  extern __shared__ __align__(16) uint8_t smb[];
+  __shared__ __align__(8) uint64_t staged;
+  const int len = H / S;                        // a multiple of 8
+  const int sl = blockIdx.x % S, g = blockIdx.x / S;
+  const int h0 = sl * len, e0 = g * kGroupE;
+  const int ne = min(kGroupE, E - e0);          // experts of this CTA
+  const int xpitch = len + 8;                   // elements; rows 16-byte aligned, banks staggered
+  const int wpitch = len + 4;                   // floats
+  float* red = reinterpret_cast<float*>(smb);   // [kLogitWarps][kGroupE][kMaxDecodeT]
+  float* ws = red + kRedFloats;                 // [kGroupE][wpitch]; rows past ne unused
+  uint8_t* xs = reinterpret_cast<uint8_t*>(ws + kGroupE * wpitch);  // [T][xpitch] of x's type
+  constexpr int eb = x_elem_bytes<XBF16>();
+  // stage the slice with one bulk copy per row, all in flight at once (rows are
+  // contiguous; every address 16-byte aligned and every size a multiple of 16:
+  // H % 64 == 0 and the pitches are multiples of 8 elements)
+  if (threadIdx.x == 0) {
+    mbar_init(&staged, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&staged, (uint32_t)(T * len * eb + ne * len * 4));
+    for (int t = 0; t < T; ++t)
+      bulk_g2s(xs + (size_t)t * xpitch * eb, static_cast<const uint8_t*>(x) + ((size_t)t * H + h0) * eb,
+               (uint32_t)(len * eb), &staged);
+    for (int el = 0; el < ne; ++el)
+      bulk_g2s(ws + (size_t)el * wpitch, Wr + (size_t)(e0 + el) * H + h0, (uint32_t)(len * 4), &staged);
+  }
+  __syncthreads();  // the barrier is initialised before anyone waits on it
+  if (!mbar_wait(&staged, 0)) {
+    if (threadIdx.x == 0) raise_flag(flags, MOE_FLAG_TIMEOUT);
+    return;
+  }
+  __syncthreads();
+  // lane tile: experts 2*(lane%4) .. +1, tokens 4*(lane/4) .. +3 (rows past T are
+  // never read: their sums stay zero and are not stored); warp w takes the K
+  // steps of 4 with index = w mod kLogitWarps, in ascending order
+  const int w = warp_id(), lane = lane_id();
+  const int ea = 2 * (lane % 4), ta = 4 * (lane / 4);
+  float acc[2][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  for (int c = 4 * w; c < len; c += 4 * kLogitWarps) {
+    float4 wv[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) wv[i] = *reinterpret_cast<const float4*>(ws + (ea + i) * wpitch + c);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (ta + j < T) {
+        float xv[4];
+        if (XBF16) {
+          const uint2 u = *reinterpret_cast<const uint2*>(xs + ((size_t)(ta + j) * xpitch + c) * 2);
+          xv[0] = bf16_to_f32(u.x & 0xFFFFu);
+          xv[1] = bf16_to_f32(u.x >> 16);
+          xv[2] = bf16_to_f32(u.y & 0xFFFFu);
+          xv[3] = bf16_to_f32(u.y >> 16);
+        } else {
+          const float4 u = *reinterpret_cast<const float4*>(xs + ((size_t)(ta + j) * xpitch + c) * 4);
+          xv[0] = u.x; xv[1] = u.y; xv[2] = u.z; xv[3] = u.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          acc[i][j] = fmaf(wv[i].x, xv[0], acc[i][j]);
+          acc[i][j] = fmaf(wv[i].y, xv[1], acc[i][j]);
+          acc[i][j] = fmaf(wv[i].z, xv[2], acc[i][j]);
+          acc[i][j] = fmaf(wv[i].w, xv[3], acc[i][j]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) red[w * (kGroupE * kMaxDecodeT) + (ea + i) * kMaxDecodeT + ta + j] = acc[i][j];
+  __syncthreads();
+  // warps in a fixed order -> partial[sl][t][e]
+  for (int i = threadIdx.x; i < kGroupE * kMaxDecodeT; i += blockDim.x) {
+    const int el = i / kMaxDecodeT, t = i % kMaxDecodeT, e = e0 + el;
+    if (t < T && e < E) {
+      float sum = 0.f;
+#pragma unroll
+      for (int ww = 0; ww < kLogitWarps; ++ww) sum += red[ww * (kGroupE * kMaxDecodeT) + i];
+      partial[((size_t)sl * T + t) * E + e] = sum;
+    }
+  }
+}
+
+template <int PER_LANE, int S>
+__global__ void __launch_bounds__(1024) topk_sort_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                         int router, const float* __restrict__ bias,
+                                                         const uint8_t* __restrict__ mask, float scale,
+                                                         int32_t* __restrict__ idx, float* __restrict__ wout,
+                                                         int chunk, int32_t* __restrict__ counts,
+                                                         int32_t* __restrict__ offsets, int32_t* __restrict__ touched,
+                                                         int32_t* __restrict__ group_base,
+                                                         int32_t* __restrict__ tile_base, int32_t* __restrict__ meta,
+                                                         int32_t* __restrict__ sorted_pair, uint32_t* flags) {
+  __shared__ int32_t base[route_dev::kSortWarps][route_dev::kSmallE];
+  __shared__ int warp_sums[32];
+  for (int t = warp_id(); t < T; t += blockDim.x >> 5)
+    route_dev::warp_topk<PER_LANE, S>(logits, T, t, E, k, router, bias, mask, scale, idx, wout, flags);
+  __syncthreads();  // the routing written above is visible to the whole block
+  route_dev::block_small_sort(idx, T * k, E, chunk, counts, offsets, touched, group_base, tile_base, meta,
+                              sorted_pair, flags, base, warp_sums);
+}
+
+}  // namespace
+
+bool decode_route_ok(const moe_desc& d, int T) { return T >= 1 && T <= 32; }
+
+bool fused_route_sort_ok(const moe_desc& d, int T) {
+  return decode_route_ok(d, T) && d.E <= route_dev::kSmallE && small_sort_ok(T * d.k, d.E);
+}
+
+static size_t decode_logits_smem(int H, int T, int S, bool xbf16) {
+  const int len = H / S;
+  return sizeof(float) * ((size_t)kRedFloats + (size_t)kGroupE * (len + 4)) + (size_t)T * (len + 8) * (xbf16 ? 2 : 4);
+}
+
+// power-of-two split of H: enough CTAs to spread the W_r stream and the FMAs
+// over most of the SMs (S x E/8 >= 128), and a slice that fits in shared
+// memory; at most 8 (the top-k templates stop there; 8 fits every H <= 8192
+// at T <= 32)
+int decode_logit_splits(const moe_desc& d, int T) {
+  const int groups = (d.E + kGroupE - 1) / kGroupE;
+  int S = 1;
+  while (S < 8 && (S * groups < 128 || decode_logits_smem(d.H, T, S, d.xfmt == MOE_X_BF16) > kLogitSmemCap))
+    S *= 2;
+  return S;
+}
+
+cudaError_t launch_decode_logits(const moe_desc& d, const void* x, int T, float* partial, int S, uint32_t* flags,
+                                 cudaStream_t s) {
+  const dim3 grid(S * ((d.E + kGroupE - 1) / kGroupE));
+  const bool xb = d.xfmt == MOE_X_BF16;
+  const size_t smem = decode_logits_smem(d.H, T, S, xb);
+  auto kern = xb ? decode_logits_kernel<true> : decode_logits_kernel<false>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  return launch_k(kern, grid, dim3(kLogitThreads), smem, s, x, d.W_r, T, d.H, d.E, S, partial, flags);
+}
+
+cudaError_t launch_topk_sort(const moe_desc& d, const float* partial, int S, int T, int32_t* idx, float* w,
+                             int chunk, const Workspace& ws, uint32_t* flags, cudaStream_t s) {
+#define MOE_TOPK_SORT(SS)                                                                                      \
+  return launch_k(topk_sort_kernel<8, SS>, dim3(1), dim3(1024), 0, s, partial, T, d.E, d.k, d.router, d.b,     \
+                  d.expert_mask, d.scale, idx, w, chunk, ws.counts, ws.offsets, ws.touched, ws.group_base,    \
+                  ws.tile_base, ws.meta, ws.sorted_pair, flags)
+  switch (S) {
+    case 1: MOE_TOPK_SORT(1);
+    case 2: MOE_TOPK_SORT(2);
+    case 4: MOE_TOPK_SORT(4);
+    default: MOE_TOPK_SORT(8);
+  }
+#undef MOE_TOPK_SORT
+}
+
+}  // namespace moe

@@ -20,6 +20,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "route_dev.cuh"
 
 namespace moe {
 
@@ -119,11 +120,6 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const void* __restri
   }
 }
 
-// (key, expert) ordering: larger key first, then smaller expert index
-__device__ __forceinline__ bool better(float ka, int ea, float kb, int eb) {
-  return ka > kb || (ka == kb && ea < eb);
-}
-
 template <int PER_LANE, int S>
 __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ partial, int T,
                                                           int E, int k, int router,
@@ -133,92 +129,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
                                                           uint32_t* flags) {
   const int t = blockIdx.x * (blockDim.x >> 5) + warp_id();
   if (t >= T) return;
-  const int lane = lane_id();
-  float logit[PER_LANE], key[PER_LANE];
-  uint32_t avail = 0;
-  bool bad = false;
-  // issue every partial load before summing (split sums in a fixed order)
-  float part[PER_LANE][S];
-#pragma unroll
-  for (int j = 0; j < PER_LANE; ++j)
-#pragma unroll
-    for (int s = 0; s < S; ++s)
-      part[j][s] = (lane + 32 * j < E) ? partial[((size_t)s * T + t) * E + lane + 32 * j] : 0.f;
-#pragma unroll
-  for (int j = 0; j < PER_LANE; ++j) {
-    const int e = lane + 32 * j;
-    logit[j] = 0.f;
-    key[j] = -INFINITY;
-    if (e < E) {
-      float l = 0.f;
-#pragma unroll
-      for (int s = 0; s < S; ++s) l += part[j][s];
-      logit[j] = l;
-      const bool active = (mask == nullptr) || (mask[e] != 0);
-      if (!isfinite(l)) {
-        bad = true;
-      } else if (active) {
-        key[j] = (router == MOE_ROUTER_SIGMOID_BIAS) ? sigmoidf_acc(l) + (bias ? bias[e] : 0.f) : l;
-        avail |= 1u << j;
-      }
-    }
-  }
-  if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) raise_flag(flags, MOE_FLAG_NONFINITE_LOGIT);
-
-  int my_e = -1;
-  float my_r = 0.f;
-  for (int slot = 0; slot < k; ++slot) {
-    float bk = -INFINITY;
-    int be = 0x7FFFFFFF;
-#pragma unroll
-    for (int j = 0; j < PER_LANE; ++j) {
-      if ((avail >> j) & 1u) {
-        const int e = lane + 32 * j;
-        if (better(key[j], e, bk, be)) {
-          bk = key[j];
-          be = e;
-        }
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ok = __shfl_xor_sync(0xFFFFFFFFu, bk, off);
-      const int oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
-      if (better(ok, oe, bk, be)) {
-        bk = ok;
-        be = oe;
-      }
-    }
-    const bool found = be != 0x7FFFFFFF;
-    float r = 0.f;
-    if (found && (be & 31) == lane) {
-      const int jj = be >> 5;
-#pragma unroll
-      for (int j = 0; j < PER_LANE; ++j)
-        if (j == jj) {
-          r = (router == MOE_ROUTER_SIGMOID_BIAS) ? sigmoidf_acc(logit[j]) : logit[j];
-          avail &= ~(1u << j);
-        }
-    }
-    r = __shfl_sync(0xFFFFFFFFu, r, found ? (be & 31) : 0);
-    if (lane == slot) {
-      my_e = found ? be : -1;
-      my_r = r;
-    }
-    if (!found && lane == 0) raise_flag(flags, MOE_FLAG_TOO_FEW_ACTIVE);
-  }
-  // renormalise over the chosen slots (softmax: exp relative to the best logit,
-  // which the full softmax denominator cancels against)
-  const float top = __shfl_sync(0xFFFFFFFFu, my_r, 0);
-  float v = 0.f;
-  if (lane < k && my_e >= 0) v = (router == MOE_ROUTER_SIGMOID_BIAS) ? my_r : expf(my_r - top);
-  float total = v;
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) total += __shfl_xor_sync(0xFFFFFFFFu, total, off);
-  if (lane < k) {
-    idx[(size_t)t * k + lane] = my_e;
-    wout[(size_t)t * k + lane] = (my_e >= 0 && total > 0.f) ? v / total * scale : 0.f;
-  }
+  route_dev::warp_topk<PER_LANE, S>(partial, T, t, E, k, router, bias, mask, scale, idx, wout, flags);
 }
 
 }  // namespace

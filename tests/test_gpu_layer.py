@@ -1,0 +1,90 @@
+"""GPU parity of moe_layer_forward: route and forward in one call, with the
+router logits, top-k and expert sort fused into two launches for decode-sized
+batches (T <= 32, E <= 256), and the separate steps otherwise."""
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_layer_31_b200 as moe
+import synth
+from gpu_util import judge, layer_from_problem, x_to_device
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "kimi-bf16-decode": (2, dict(T=32, H=256, E=64, I=256)),
+    "kimi-bf16-T1": (2, dict(T=1, H=256, E=64, I=128)),
+    "kimi-bf16-T7-ragged": (2, dict(T=7, H=320, E=40, I=192)),
+    "kimi-int8-decode": (3, dict(T=24, H=384, E=48, I=256)),
+    "qwen3-int4-softmax": (4, dict(T=32, H=256, E=128, I=128)),
+    "tiny-fp32": (1, {}),
+    "skew-masked": (5, dict(T=30, H=256, E=64, I=128, n_active=20, bias=("skew", 0.2))),
+    "wide-E-fallback": (2, dict(T=16, H=256, E=320, I=128)),
+    "T33-fallback": (3, dict(T=33, H=256, E=32, I=128)),
+    "gelu-int4b128": (4, dict(T=20, H=256, E=32, I=256, wfmt="int4b128", act="gelu_tanh")),
+}
+
+
+@pytest.fixture(autouse=True)
+def _clear_flags():
+    moe.moe_device_flags(clear=True)
+    yield
+    assert moe.moe_device_flags(clear=True) == 0
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_layer_forward_matches_oracle_and_the_separate_steps(name):
+    cid, over = CASES[name]
+    prob = synth.make_problem(cid, **over)
+    layer = layer_from_problem(prob)
+    x = x_to_device(prob)
+    y, idx, w = layer.layer(x)
+    torch.cuda.synchronize()
+    judge(prob, y, idx, w)
+    # the separate entry points on the same input: same routing, same output, bit for bit
+    i2, w2 = layer.route(x)
+    y2 = layer.forward(x, i2, w2)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, i2) and torch.equal(w, w2)
+    assert torch.equal(y.view(torch.int16) if y.dtype == torch.bfloat16 else y,
+                       y2.view(torch.int16) if y2.dtype == torch.bfloat16 else y2)
+
+
+def test_layer_forward_full_decode_shape():
+    prob = synth.make_problem(2)
+    layer = layer_from_problem(prob)
+    y, idx, w = layer.layer(x_to_device(prob))
+    torch.cuda.synchronize()
+    judge(prob, y, idx, w)
+
+
+def test_decode_router_mask_equals_slice():
+    """The decode logits kernel keeps masking experts equal to slicing them, bit for bit."""
+    prob = synth.make_problem(5, T=32, H=256, E=48, I=128, n_active=29, bias=("skew", 0.2))
+    act = np.nonzero(prob.mask)[0]
+    sl = synth.Problem(cfg=prob.cfg, T=prob.T, H=prob.H, I=prob.I, E=len(act), k=prob.k, router=prob.router,
+                       scale=prob.scale, wfmt=prob.wfmt, xfmt=prob.xfmt, x=prob.x,
+                       W_r=np.ascontiguousarray(prob.W_r[act]), b=np.ascontiguousarray(prob.b[act]), mask=None,
+                       W_gate=np.ascontiguousarray(prob.W_gate[act]), W_up=np.ascontiguousarray(prob.W_up[act]),
+                       W_down=np.ascontiguousarray(prob.W_down[act]), s_gate=np.ascontiguousarray(prob.s_gate[act]),
+                       s_up=np.ascontiguousarray(prob.s_up[act]), s_down=np.ascontiguousarray(prob.s_down[act]))
+    y1, i1, w1 = layer_from_problem(prob).layer(x_to_device(prob))
+    y2, i2, w2 = layer_from_problem(sl).layer(x_to_device(sl))
+    torch.cuda.synchronize()
+    assert np.array_equal(act[i2.cpu().numpy()], i1.cpu().numpy())
+    assert torch.equal(w1, w2)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+def test_layer_forward_launches_fewer_kernels_at_decode():
+    prob = synth.make_problem(2, T=32, H=256, E=64, I=128)
+    layer = layer_from_problem(prob)
+    x = x_to_device(prob)
+    layer.layer(x)
+    n0 = moe.moe_launch_count()
+    layer.layer(x)
+    fused = moe.moe_launch_count() - n0
+    n0 = moe.moe_launch_count()
+    layer(x)
+    separate = moe.moe_launch_count() - n0
+    assert fused == separate - 1  # top-k and sort share one launch

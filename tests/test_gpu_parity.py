@@ -194,9 +194,9 @@ def test_zero_tokens_is_a_noop():
     assert moe.moe_launch_count() == n
 
 
-@pytest.mark.parametrize("cid", [1, 2])
-def test_stage_timing_reports_every_kernel(cid):
-    prob = synth.make_problem(cid, T=16, H=256, E=16, I=128)
+@pytest.mark.parametrize("cid,T", [(1, 16), (2, 16), (1, 40), (2, 40)])
+def test_stage_timing_reports_every_kernel(cid, T):
+    prob = synth.make_problem(cid, T=T, H=256, E=16, I=128)
     layer = layer_from_problem(prob)
     x = x_to_device(prob)
     moe.moe_stage_timing(True)
@@ -205,7 +205,10 @@ def test_stage_timing_reports_every_kernel(cid):
         times = moe.moe_stage_times()
     finally:
         moe.moe_stage_timing(False)
-    router = ("router_split3", "router_logits_tc") if prob.xfmt == "bf16" else ("router_logits",)
+    if T <= 32:
+        router = ("router_decode_logits",)
+    else:
+        router = ("router_split3", "router_logits_tc") if prob.xfmt == "bf16" else ("router_logits",)
     for name in router + ("router_topk", "combine"):
         assert name in times and times[name][0] == 1 and times[name][1] > 0
     sort = ("small_sort",) if "small_sort" in times else ("pair_histogram", "expert_scan", "pair_scatter")
