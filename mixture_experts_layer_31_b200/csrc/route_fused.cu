@@ -136,8 +136,18 @@ __global__ void __launch_bounds__(kLogitThreads) decode_logits_kernel(const void
   }
 }
 
+// One CTA of 1024 threads, three phases with one global round trip:
+//   A  every thread sums the S partial logits of some (token, expert) pairs in
+//      the split order (split 0 first, as the standalone top-k does) into
+//      shared memory, and the bias and mask are staged there;
+//   B  one warp per token selects its top-k from shared memory (the same device
+//      code as the standalone top-k, so the routing is bit for bit the same);
+//   C  the stable counting sort reads the routing from shared memory.
+// The logits and the sort's per-warp bases share one buffer (never live together).
+constexpr int kFusedMaxT = 32, kFusedMaxE = 256, kFusedMaxK = 32;
+
 template <int PER_LANE, int S>
-__global__ void __launch_bounds__(1024) topk_sort_kernel(const float* __restrict__ logits, int T, int E, int k,
+__global__ void __launch_bounds__(1024) topk_sort_kernel(const float* __restrict__ partial, int T, int E, int k,
                                                          int router, const float* __restrict__ bias,
                                                          const uint8_t* __restrict__ mask, float scale,
                                                          int32_t* __restrict__ idx, float* __restrict__ wout,
@@ -146,13 +156,37 @@ __global__ void __launch_bounds__(1024) topk_sort_kernel(const float* __restrict
                                                          int32_t* __restrict__ group_base,
                                                          int32_t* __restrict__ tile_base, int32_t* __restrict__ meta,
                                                          int32_t* __restrict__ sorted_pair, uint32_t* flags) {
-  __shared__ int32_t base[route_dev::kSortWarps][route_dev::kSmallE];
+  static_assert(kFusedMaxT * kFusedMaxE == route_dev::kSortWarps * route_dev::kSmallE, "shared buffer sizes");
+  __shared__ __align__(16) int32_t buf[route_dev::kSortWarps][route_dev::kSmallE];  // logits, then sort bases
+  __shared__ float bias_s[kFusedMaxE];
+  __shared__ uint8_t mask_s[kFusedMaxE];
+  __shared__ int32_t idx_s[kFusedMaxT * kFusedMaxK];
   __shared__ int warp_sums[32];
+  float* logits = reinterpret_cast<float*>(&buf[0][0]);  // [T][E]
+  // A: partial sums, all loads of a thread in flight together
+  for (int i = threadIdx.x; i < T * E; i += blockDim.x) {
+    const int t = i / E, e = i - t * E;
+    float p[S];
+#pragma unroll
+    for (int s = 0; s < S; ++s) p[s] = partial[((size_t)s * T + t) * E + e];
+    float sum = 0.f;
+#pragma unroll
+    for (int s = 0; s < S; ++s) sum += p[s];
+    logits[i] = sum;
+  }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    if (bias) bias_s[e] = bias[e];
+    if (mask) mask_s[e] = mask[e];
+  }
+  __syncthreads();
+  // B
   for (int t = warp_id(); t < T; t += blockDim.x >> 5)
-    route_dev::warp_topk<PER_LANE, S>(logits, T, t, E, k, router, bias, mask, scale, idx, wout, flags);
-  __syncthreads();  // the routing written above is visible to the whole block
-  route_dev::block_small_sort(idx, T * k, E, chunk, counts, offsets, touched, group_base, tile_base, meta,
-                              sorted_pair, flags, base, warp_sums);
+    route_dev::warp_topk<PER_LANE, 1>(logits, T, t, E, k, router, bias ? bias_s : nullptr, mask ? mask_s : nullptr,
+                                      scale, idx, wout, flags, idx_s);
+  __syncthreads();
+  // C
+  route_dev::block_small_sort(idx_s, T * k, E, chunk, counts, offsets, touched, group_base, tile_base, meta,
+                              sorted_pair, flags, buf, warp_sums);
 }
 
 }  // namespace
@@ -160,7 +194,8 @@ __global__ void __launch_bounds__(1024) topk_sort_kernel(const float* __restrict
 bool decode_route_ok(const moe_desc& d, int T) { return T >= 1 && T <= 32; }
 
 bool fused_route_sort_ok(const moe_desc& d, int T) {
-  return decode_route_ok(d, T) && d.E <= route_dev::kSmallE && small_sort_ok(T * d.k, d.E);
+  return decode_route_ok(d, T) && T <= kFusedMaxT && d.E <= kFusedMaxE && d.k <= kFusedMaxK &&
+         small_sort_ok(T * d.k, d.E);
 }
 
 static size_t decode_logits_smem(int H, int T, int S, bool xbf16) {
