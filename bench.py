@@ -182,9 +182,16 @@ def algorithmic(prob, idx: np.ndarray):
     layer_bytes = ut * (gate_up_per_expert + down_per_expert) + prob.W_r.nbytes + 2 * T * H * xb
     layer_flops = 6.0 * P * H * I + 2.0 * T * H * E
     if prob.I_s:  # the block: shared expert weights (+ scales) and flops, residual read
-        layer_bytes += sum(a.nbytes for a in (prob.Ws_gate, prob.Ws_up, prob.Ws_down, prob.ss_gate, prob.ss_up,
-                                              prob.ss_down) if a is not None)
+        sh = lambda W, S: W.nbytes + (0 if S is None else S.nbytes)
+        sh_up = sh(prob.Ws_gate, prob.ss_gate) + sh(prob.Ws_up, prob.ss_up)
+        sh_down = sh(prob.Ws_down, prob.ss_down)
+        layer_bytes += sh_up + sh_down
         layer_flops += 6.0 * T * H * prob.I_s
+        # on the tensor-core path the shared expert's units run inside the routed launches
+        bytes_["gemm_gateup"] += sh_up + T * H * 2 + T * prob.I_s * 2
+        bytes_["gemm_down"] += sh_down + T * prob.I_s * 2 + T * H * 4
+        flops["gemm_gateup"] += 4.0 * T * H * prob.I_s
+        flops["gemm_down"] += 2.0 * T * H * prob.I_s
     if prob.residual is not None:
         layer_bytes += T * H * xb
     return dict(touched=ut, per_expert_gate_up=gate_up_per_expert, per_expert_down=down_per_expert, bytes=bytes_,

@@ -79,6 +79,14 @@ struct GemmArgs {
   int Hx;               // columns of x (the K coordinate of x is taken modulo Hx)
   int act;              // gate/up: moe_act (SiLU or tanh-GELU)
   int qsh;              // int4: log2 of the scale block (5: 32 columns, 7: 128)
+  // optional second, dense problem in the same launch (the shared expert): every
+  // one of Td tokens in token order with weight 1, expert 0 of weights with Rd rows
+  // and Kd columns; its units follow the routed ones
+  int dense_units;      // 0: none
+  int Rd, Kd, Td, chunkd;
+  const float* sd0;
+  const float* sd1;
+  void* outd;           // gate/up: h [Td, Rd] bf16; down: rows [Td, Rd] fp32
 };
 
 __device__ __forceinline__ void wait_or_die(uint64_t* bar, uint32_t parity, bool& dead, uint32_t* flags) {
@@ -92,14 +100,46 @@ __device__ __forceinline__ void wait_or_die(uint64_t* bar, uint32_t parity, bool
 struct Unit {
   int e, base, ib, c, n_tok, n_mma;
   int k0, nk;  // K steps [k0, k0 + nk)
+  int pos0;    // first sorted position (dense: first token) of the unit's chunk
+  bool dense;  // a unit of the dense problem
 };
+
+// The per-problem view a role needs for a unit.
+struct ProbView {
+  int R, K;
+  const float* s0;
+  const float* s1;
+  void* out;
+};
+
+__device__ __forceinline__ ProbView view_of(const GemmArgs& a, const Unit& t) {
+  if (t.dense) return ProbView{a.Rd, a.Kd, a.sd0, a.sd1, a.outd};
+  return ProbView{a.R, a.K, a.s0, a.s1, a.out};
+}
 
 // units of the expert GEMMs (MODE 0/1): (expert, output-row block, token chunk),
 // chunks fastest; of the router GEMM (MODE 2): (token chunk, expert block, K split)
 template <int MODE>
-__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u, int nib, int ntouched) {
+__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u, int nib, int ntouched, int routed) {
   Unit t;
   const int nk_all = a.K / kBK;
+  t.dense = false;
+  if (MODE != 2 && u >= routed) {
+    // dense problem: (row block, token chunk), chunks fastest
+    const int v = u - routed;
+    const int nc = (a.Td + a.chunkd - 1) / a.chunkd;
+    t.dense = true;
+    t.e = 0;
+    t.base = 0;
+    t.ib = v / nc;
+    t.c = v - t.ib * nc;
+    t.pos0 = t.c * a.chunkd;
+    t.n_tok = min(a.chunkd, a.Td - t.pos0);
+    t.n_mma = (t.n_tok + 15) & ~15;
+    t.k0 = 0;
+    t.nk = a.Kd / kBK;
+    return t;
+  }
   if (MODE == 2) {
     const int s = u % a.S, r = u / a.S;
     t.ib = r % nib;
@@ -110,6 +150,7 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u, int nib, i
     t.n_mma = (t.n_tok + 15) & ~15;
     t.k0 = s * nk_all / a.S;
     t.nk = (s + 1) * nk_all / a.S - t.k0;
+    t.pos0 = t.base;
     return t;
   }
   int lo = 0, hi = ntouched - 1;
@@ -129,6 +170,7 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u, int nib, i
   t.n_mma = (t.n_tok + 15) & ~15;
   t.k0 = 0;
   t.nk = nk_all;
+  t.pos0 = t.base + t.c * a.chunk;
   return t;
 }
 
@@ -190,7 +232,9 @@ struct Traits {
 template <int MODE, int WF, int MT>
 __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
-                   const __grid_constant__ CUtensorMap tm_b, const GemmArgs a) {
+                   const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_w0d,
+                   const __grid_constant__ CUtensorMap tm_w1d, const __grid_constant__ CUtensorMap tm_bd,
+                   const GemmArgs a) {
   using Tr = Traits<MODE, WF, MT>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -238,6 +282,11 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
     prefetch_tmap(&tm_w0);
     if (MODE == 0) prefetch_tmap(&tm_w1);
     prefetch_tmap(&tm_b);
+    if (a.dense_units > 0) {
+      prefetch_tmap(&tm_w0d);
+      if (MODE == 0) prefetch_tmap(&tm_w1d);
+      prefetch_tmap(&tm_bd);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -246,8 +295,9 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
 
   const int ntouched = MODE == 2 ? 0 : a.meta[0];
   const int nib = (a.R + Tr::kRows - 1) / Tr::kRows;  // gate/up: the last block may be half (I % 128 == 64)
-  const int total = MODE == 2 ? nib * ((a.T + a.chunk - 1) / a.chunk) * a.S
-                              : (ntouched > 0 ? a.meta[3] * nib : 0);
+  const int routed = MODE == 2 ? nib * ((a.T + a.chunk - 1) / a.chunk) * a.S
+                               : (ntouched > 0 ? a.meta[3] * nib : 0);
+  const int total = routed + (MODE == 2 ? 0 : a.dense_units);
 
   if (w == 0 || (Tr::kQuant && w == 2)) {
     // ------------------------------------------------------------------ TMA producers
@@ -263,10 +313,13 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
       uint32_t it = 0;
       const uint32_t abytes = load_a ? MT * (Tr::kQuant ? Tr::kRawTile : kTileBytes) : 0;
       for (int u = blockIdx.x; u < total; u += gridDim.x) {
-        const Unit t = decode_unit<MODE>(a, u, nib, ntouched);
+        const Unit t = decode_unit<MODE>(a, u, nib, ntouched, routed);
         const int nbox = load_b ? (t.n_tok + kBoxRows - 1) / kBoxRows : 0;
-        const int brow = MODE == 2 ? t.base : t.base + t.c * a.chunk;
-        const int wrow0 = t.e * a.R + t.ib * Tr::kRows;
+        const int brow = t.pos0;
+        const int wrow0 = t.e * (t.dense ? a.Rd : a.R) + t.ib * Tr::kRows;
+        const CUtensorMap* mw0 = t.dense ? &tm_w0d : &tm_w0;
+        const CUtensorMap* mw1 = t.dense ? &tm_w1d : &tm_w1;
+        const CUtensorMap* mb = t.dense ? &tm_bd : &tm_b;
         for (int kb = t.k0; kb < t.k0 + t.nk; ++kb, ++it) {
           const int s = it % ring;
           wait_or_die(&re[s], ((it / ring) & 1u) ^ 1u, dead, a.flags);
@@ -279,16 +332,16 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
             for (int mt = 0; mt < MT; ++mt) {
               uint8_t* adst = ad + mt * (Tr::kQuant ? Tr::kRawTile : kTileBytes);
               if (MODE == 0)  // tile 0: 128 gate rows, tile 1: the same 128 up rows
-                tma_load_2d(adst, mt ? &tm_w1 : &tm_w0, wcol, wrow0, &rf[s]);
+                tma_load_2d(adst, mt ? mw1 : mw0, wcol, wrow0, &rf[s]);
               else            // 128 down rows per tile
-                tma_load_2d(adst, &tm_w0, wcol, wrow0 + mt * kBM, &rf[s]);
+                tma_load_2d(adst, mw0, wcol, wrow0 + mt * kBM, &rf[s]);
             }
           }
           if (load_b) {
             uint8_t* st = stages + (size_t)s * a.stage_bytes;
             const int bcol = MODE == 2 ? (kb * kBK) % a.Hx : kb * kBK;
             for (int j = 0; j < nbox; ++j)
-              tma_load_2d(st + a.b_off + j * kBoxRows * kBK * 2, &tm_b, bcol, brow + kBoxRows * j, &rf[s]);
+              tma_load_2d(st + a.b_off + j * kBoxRows * kBK * 2, mb, bcol, brow + kBoxRows * j, &rf[s]);
           }
         }
       }
@@ -304,7 +357,7 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
       const uint32_t stage0 = smem_u32(stages);
       const uint32_t a_ring0 = smem_u32(a_ring);
       for (int u = blockIdx.x; u < total; u += gridDim.x, ++local) {
-        const Unit t = decode_unit<MODE>(a, u, nib, ntouched);
+        const Unit t = decode_unit<MODE>(a, u, nib, ntouched, routed);
         const uint32_t buf = local % nbuf;
         wait_or_die(&acc_empty[buf], ((local / nbuf) & 1u) ^ 1u, dead, a.flags);
         tc_fence_after();
@@ -350,7 +403,7 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
     bool dead = false;
     uint32_t local = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x, ++local) {
-      const Unit t = decode_unit<MODE>(a, u, nib, ntouched);
+      const Unit t = decode_unit<MODE>(a, u, nib, ntouched, routed);
       const uint32_t buf = local % nbuf;
       if (lane == 0) wait_or_die(&acc_full[buf], (local / nbuf) & 1u, dead, a.flags);
       if (MODE != 1) {
@@ -362,16 +415,17 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
       tc_fence_after();
       const int tile = split_cols ? 0 : grp;
       const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * buf_cols + tile * a.acc_stride;
-      const int pos0 = t.base + t.c * a.chunk;
+      const int pos0 = t.pos0;
+      const ProbView pv = view_of(a, t);
       const int c_first = split_cols ? grp * 16 : 0, c_step = split_cols ? 32 : 16;
       if (!dead) {
         if (MODE == 0) {
           const int row = t.ib * kBM + q * 32 + lane;
-          const bool live = row < a.R;
-          const size_t grow = (size_t)t.e * a.R + (live ? row : 0);
-          const float sg = WF == MOE_W_INT8_ROW ? a.s0[grow] : 1.f;
-          const float su = WF == MOE_W_INT8_ROW ? a.s1[grow] : 1.f;
-          uint16_t* hout = static_cast<uint16_t*>(a.out);
+          const bool live = row < pv.R;
+          const size_t grow = (size_t)t.e * pv.R + (live ? row : 0);
+          const float sg = WF == MOE_W_INT8_ROW ? pv.s0[grow] : 1.f;
+          const float su = WF == MOE_W_INT8_ROW ? pv.s1[grow] : 1.f;
+          uint16_t* hout = static_cast<uint16_t*>(pv.out);
           for (int n0 = c_first; n0 < t.n_tok; n0 += c_step) {
             uint32_t g[16], v[16];
             tmem_ld16(tacc + n0, g);
@@ -383,7 +437,7 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
                 if (n0 + j < t.n_tok) {
                   const float gv = __uint_as_float(g[j]) * sg, uv = __uint_as_float(v[j]) * su;
                   const float hv = a.act == MOE_ACT_GELU_TANH ? gelu_tanh_mul_fast(gv, uv) : silu_mul_fast(gv, uv);
-                  hout[(size_t)(pos0 + n0 + j) * a.R + row] = f32_to_bf16(hv);
+                  hout[(size_t)(pos0 + n0 + j) * pv.R + row] = f32_to_bf16(hv);
                 }
               }
             }
@@ -408,14 +462,15 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
           float* s_w = gx + 256;
           const int et = q * 32 + lane;
           for (int n = et; n < t.n_tok; n += 128) {
-            const int pair = a.sorted_pair[pos0 + n];
+            // dense problem: the token itself, weight 1
+            const int pair = t.dense ? pos0 + n : a.sorted_pair[pos0 + n];
             s_pair[n] = pair;
-            s_w[n] = a.topk_w[pair];
+            s_w[n] = t.dense ? 1.f : a.topk_w[pair];
           }
           named_bar_sync(bar_x, 128);
           const int row = t.ib * Tr::kRows + tile * kBM + et;
-          const float sd = WF == MOE_W_INT8_ROW ? a.s0[(size_t)t.e * a.R + row] : 1.f;
-          float* yp = static_cast<float*>(a.out);
+          const float sd = WF == MOE_W_INT8_ROW ? pv.s0[(size_t)t.e * pv.R + row] : 1.f;
+          float* yp = static_cast<float*>(pv.out);
           for (int n0 = c_first; n0 < t.n_tok; n0 += c_step) {
             uint32_t v[16];
             tmem_ld16(tacc + n0, v);
@@ -423,7 +478,7 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               if (n0 + j < t.n_tok)
-                yp[(size_t)s_pair[n0 + j] * a.R + row] = s_w[n0 + j] * sd * __uint_as_float(v[j]);
+                yp[(size_t)s_pair[n0 + j] * pv.R + row] = s_w[n0 + j] * sd * __uint_as_float(v[j]);
             }
           }
         }
@@ -444,18 +499,19 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
     bool dead = false;
     uint32_t it = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
-      const Unit t = decode_unit<MODE>(a, u, nib, ntouched);
+      const Unit t = decode_unit<MODE>(a, u, nib, ntouched, routed);
       // int4: block scales of this thread's rows, one K step ahead
+      const ProbView pv = view_of(a, t);
       const float* srow[kPer];
       float sc_next[kPer];
 #pragma unroll
       for (int j = 0; j < kPer; ++j) {
         const int r = r0 + kRowStep * j;  // row within the unit's MT*128 A rows
         const int mt = r >> 7, rr = r & 127;
-        const float* S = (MODE == 0 && mt == 1) ? a.s1 : a.s0;
+        const float* S = (MODE == 0 && mt == 1) ? pv.s1 : pv.s0;
         int wr = MODE == 0 ? t.ib * kBM + rr : t.ib * Tr::kRows + mt * kBM + rr;
-        if (wr >= a.R) wr = a.R - 1;  // rows past a half block are computed but never stored
-        srow[j] = S + ((size_t)t.e * a.R + wr) * (a.K >> a.qsh);
+        if (wr >= pv.R) wr = pv.R - 1;  // rows past a half block are computed but never stored
+        srow[j] = S + ((size_t)t.e * pv.R + wr) * (pv.K >> a.qsh);
         sc_next[j] = WF == MOE_W_INT4_B32 ? __ldg(srow[j] + ((t.k0 * kBK + c8 * 8) >> a.qsh)) : 1.f;
       }
       for (int kb = 0; kb < t.nk; ++kb, ++it) {
@@ -553,19 +609,27 @@ uint32_t pow2_at_least(uint32_t v) {
   return p;
 }
 
+// tensor maps of one launch: the routed problem's weights and token rows, and
+// the dense problem's (copies of the routed ones when there is none)
+struct Maps {
+  CUtensorMap w0, w1, b, w0d, w1d, bd;
+};
+
 template <int MODE, int WF, int MT>
-cudaError_t launch_gemm(const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb, GemmArgs a,
-                        int num_sms, cudaStream_t s) {
+cudaError_t launch_gemm(const Maps& m, GemmArgs a, int num_sms, cudaStream_t s) {
   using Tr = Traits<MODE, WF, MT>;
+  // the dense problem's units: (row block of Tr::kRows, token chunk)
+  a.dense_units = a.Td > 0 ? ((a.Rd + Tr::kRows - 1) / Tr::kRows) * ((a.Td + a.chunkd - 1) / a.chunkd) : 0;
+  const int chunk_max = a.dense_units > 0 && a.chunkd > a.chunk ? a.chunkd : a.chunk;
   // stage: bf16 weights [A: MT x 16 KB][B]; quantised [B], with the raw tiles in a ring of
   // their own after the main ring (their bf16 A lives in the A ring).  Token boxes are
   // kBoxRows tall: B holds the chunk rounded up to whole boxes.  All sizes are multiples of
   // 1024 (4 KB boxes, 16/8/4 KB tiles).
-  const int b_rows = (a.chunk + kBoxRows - 1) / kBoxRows * kBoxRows;
+  const int b_rows = (chunk_max + kBoxRows - 1) / kBoxRows * kBoxRows;
   a.b_off = Tr::kQuant ? 0 : MT * kTileBytes;
   a.stage_bytes = a.b_off + b_rows * kBK * 2;
   a.raw_stage_bytes = MT * Tr::kRawTile;
-  a.acc_stride = (int)pow2_at_least((uint32_t)a.chunk);
+  a.acc_stride = (int)pow2_at_least((uint32_t)chunk_max);
   a.nbuf = 2 * MT * a.acc_stride <= 512 ? 2 : 1;
   a.tmem_cols = a.nbuf * MT * a.acc_stride;
   const int fixed = 1024 + kBarrierBytes + Tr::kXchg + (Tr::kQuant ? kAStages * MT * kTileBytes : 0);
@@ -590,7 +654,7 @@ cudaError_t launch_gemm(const CUtensorMap& m0, const CUtensorMap& m1, const CUte
   auto kern = gemm_tc_kernel<MODE, WF, MT>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  return launch_k(kern, dim3(num_sms), dim3(Tr::kThreads), smem, s, m0, m1, mb, a);
+  return launch_k(kern, dim3(num_sms), dim3(Tr::kThreads), smem, s, m.w0, m.w1, m.b, m.w0d, m.w1d, m.bd, a);
 }
 
 // gate/up always carries two M tiles (gate, up); down carries two 128-row tiles
@@ -599,19 +663,17 @@ cudaError_t launch_gemm(const CUtensorMap& m0, const CUtensorMap& m1, const CUte
 // 16 KB tile per stage about 86%; at prefill sizes the token tile feeds 256
 // weight rows)
 template <int MODE>
-cudaError_t launch_by_format(int wfmt, const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& mb,
-                             const GemmArgs& a, int num_sms, cudaStream_t s) {
-  const bool two = MODE == 0 || a.R % (2 * kBM) == 0;
+cudaError_t launch_by_format(int wfmt, const Maps& m, const GemmArgs& a, int num_sms, cudaStream_t s) {
+  const bool two = MODE == 0 || a.R % (2 * kBM) == 0;  // down: the dense problem has the same R (= H)
   switch (wfmt) {
     case MOE_W_BF16:
-      return two ? launch_gemm<MODE, MOE_W_BF16, 2>(m0, m1, mb, a, num_sms, s)
-                 : launch_gemm<MODE, MOE_W_BF16, 1>(m0, m1, mb, a, num_sms, s);
+      return two ? launch_gemm<MODE, MOE_W_BF16, 2>(m, a, num_sms, s) : launch_gemm<MODE, MOE_W_BF16, 1>(m, a, num_sms, s);
     case MOE_W_INT8_ROW:
-      return two ? launch_gemm<MODE, MOE_W_INT8_ROW, 2>(m0, m1, mb, a, num_sms, s)
-                 : launch_gemm<MODE, MOE_W_INT8_ROW, 1>(m0, m1, mb, a, num_sms, s);
+      return two ? launch_gemm<MODE, MOE_W_INT8_ROW, 2>(m, a, num_sms, s)
+                 : launch_gemm<MODE, MOE_W_INT8_ROW, 1>(m, a, num_sms, s);
     default:
-      return two ? launch_gemm<MODE, MOE_W_INT4_B32, 2>(m0, m1, mb, a, num_sms, s)
-                 : launch_gemm<MODE, MOE_W_INT4_B32, 1>(m0, m1, mb, a, num_sms, s);
+      return two ? launch_gemm<MODE, MOE_W_INT4_B32, 2>(m, a, num_sms, s)
+                 : launch_gemm<MODE, MOE_W_INT4_B32, 1>(m, a, num_sms, s);
   }
 }
 
@@ -713,7 +775,8 @@ cudaError_t launch_router_tc(const moe_desc& d, const void* x, int T, const void
   a.T = T;
   a.S = S;
   a.Hx = d.H;
-  return launch_gemm<2, MOE_W_BF16, 1>(ma, ma, mb, a, num_sms, s);
+  const Maps m{ma, ma, mb, ma, ma, mb};
+  return launch_gemm<2, MOE_W_BF16, 1>(m, a, num_sms, s);
 }
 
 // gate/up tiles 128 output rows of I (a multiple of 64; a half block is computed
@@ -734,12 +797,12 @@ cudaError_t launch_gather_rows(const moe_desc& d, const void* x, const Workspace
 }
 
 cudaError_t launch_gemm_gateup(const moe_desc& d, const Workspace& ws, int P, int chunk, int num_sms,
-                               uint32_t* flags, cudaStream_t s) {
-  CUtensorMap mg, mu, mb;
-  cudaError_t e = weight_map(&mg, d.W_gate, d.wfmt, d.E, d.I, d.H, kBM);
-  if (e == cudaSuccess) e = weight_map(&mu, d.W_up, d.wfmt, d.E, d.I, d.H, kBM);
+                               uint32_t* flags, cudaStream_t s, const DenseGemm* dg) {
+  Maps m;
+  cudaError_t e = weight_map(&m.w0, d.W_gate, d.wfmt, d.E, d.I, d.H, kBM);
+  if (e == cudaSuccess) e = weight_map(&m.w1, d.W_up, d.wfmt, d.E, d.I, d.H, kBM);
   if (e == cudaSuccess)
-    e = make_map(&mb, ws.xs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.H, (uint64_t)P, kBK, kBoxRows,
+    e = make_map(&m.b, ws.xs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.H, (uint64_t)P, kBK, kBoxRows,
                  CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   GemmArgs a = common(ws, chunk, flags);
@@ -750,15 +813,34 @@ cudaError_t launch_gemm_gateup(const moe_desc& d, const Workspace& ws, int P, in
   a.K = d.H;
   a.act = d.act;
   a.qsh = d.wfmt == MOE_W_INT4_B128 ? 7 : 5;
-  return launch_by_format<0>(d.wfmt, mg, mu, mb, a, num_sms, s);
+  m.w0d = m.w0;
+  m.w1d = m.w1;
+  m.bd = m.b;
+  if (dg) {  // the dense problem: its gate/up weights against the token rows in order
+    const moe_desc& sd = *dg->d;
+    e = weight_map(&m.w0d, sd.W_gate, sd.wfmt, 1, sd.I, sd.H, kBM);
+    if (e == cudaSuccess) e = weight_map(&m.w1d, sd.W_up, sd.wfmt, 1, sd.I, sd.H, kBM);
+    if (e == cudaSuccess)
+      e = make_map(&m.bd, dg->b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sd.H, (uint64_t)dg->T, kBK, kBoxRows,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    a.Rd = sd.I;
+    a.Kd = sd.H;
+    a.Td = dg->T;
+    a.chunkd = dg->chunk;
+    a.sd0 = sd.s_gate;
+    a.sd1 = sd.s_up;
+    a.outd = dg->out;
+  }
+  return launch_by_format<0>(d.wfmt, m, a, num_sms, s);
 }
 
 cudaError_t launch_gemm_down(const moe_desc& d, const float* topk_w, const Workspace& ws, int P, int chunk,
-                             int num_sms, uint32_t* flags, cudaStream_t s) {
-  CUtensorMap md, mb;
-  cudaError_t e = weight_map(&md, d.W_down, d.wfmt, d.E, d.H, d.I, 128);
+                             int num_sms, uint32_t* flags, cudaStream_t s, const DenseGemm* dg) {
+  Maps m;
+  cudaError_t e = weight_map(&m.w0, d.W_down, d.wfmt, d.E, d.H, d.I, 128);
   if (e == cudaSuccess)
-    e = make_map(&mb, ws.hbuf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.I, (uint64_t)P, kBK, kBoxRows,
+    e = make_map(&m.b, ws.hbuf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.I, (uint64_t)P, kBK, kBoxRows,
                  CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   GemmArgs a = common(ws, chunk, flags);
@@ -768,7 +850,26 @@ cudaError_t launch_gemm_down(const moe_desc& d, const float* topk_w, const Works
   a.R = d.H;
   a.K = d.I;
   a.qsh = d.wfmt == MOE_W_INT4_B128 ? 7 : 5;
-  return launch_by_format<1>(d.wfmt, md, md, mb, a, num_sms, s);
+  m.w1 = m.w0;
+  m.w0d = m.w0;
+  m.w1d = m.w0;
+  m.bd = m.b;
+  if (dg) {  // the dense problem: its down weights against its h rows in token order
+    const moe_desc& sd = *dg->d;
+    e = weight_map(&m.w0d, sd.W_down, sd.wfmt, 1, sd.H, sd.I, 128);
+    if (e == cudaSuccess)
+      e = make_map(&m.bd, dg->b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sd.I, (uint64_t)dg->T, kBK, kBoxRows,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    m.w1d = m.w0d;
+    a.Rd = sd.H;
+    a.Kd = sd.I;
+    a.Td = dg->T;
+    a.chunkd = dg->chunk;
+    a.sd0 = sd.s_down;
+    a.outd = dg->out;
+  }
+  return launch_by_format<1>(d.wfmt, m, a, num_sms, s);
 }
 
 }  // namespace moe

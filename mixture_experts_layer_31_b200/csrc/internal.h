@@ -99,10 +99,21 @@ cudaError_t launch_router_tc(const moe_desc& d, const void* x, int T, const void
                              int num_sms, uint32_t* flags, cudaStream_t s);
 cudaError_t launch_gather_rows(const moe_desc& d, const void* x, const Workspace& ws, int P, int num_sms,
                                cudaStream_t s);
+// An optional second, dense problem run in the same grouped-GEMM launch (the
+// shared expert): the one-expert layer *d applied to T token rows in order with
+// weight 1; b = its input rows (gate/up: x [T, H]; down: its h [T, I]), out = its
+// output rows (gate/up: h [T, I] bf16; down: [T, H] fp32); chunk its token chunk.
+struct DenseGemm {
+  const moe_desc* d;
+  const void* b;
+  void* out;
+  int T;
+  int chunk;
+};
 cudaError_t launch_gemm_gateup(const moe_desc& d, const Workspace& ws, int P, int chunk, int num_sms,
-                               uint32_t* flags, cudaStream_t s);
+                               uint32_t* flags, cudaStream_t s, const DenseGemm* dg = nullptr);
 cudaError_t launch_gemm_down(const moe_desc& d, const float* topk_w, const Workspace& ws, int P, int chunk,
-                             int num_sms, uint32_t* flags, cudaStream_t s);
+                             int num_sms, uint32_t* flags, cudaStream_t s, const DenseGemm* dg = nullptr);
 // decode-sized batches (T <= 32): fp32 logits in one launch; with E <= 256 and
 // T*k <= 8192 also top-k and the expert sort in one launch
 bool decode_route_ok(const moe_desc& d, int T);

@@ -296,7 +296,8 @@ extern "C" moe_status moe_route(const moe_desc* d, const void* x, int32_t T, int
 // leaves w * FFN rows in ws.yp
 static moe_status run_routed(const moe_desc* d, const void* x, int32_t T, const int32_t* topk_idx,
                              const float* topk_w, const Workspace& ws, int path, DeviceState* dev,
-                             cudaStream_t stream, bool sorted = false) {
+                             cudaStream_t stream, bool sorted = false, const DenseGemm* dense_up = nullptr,
+                             const DenseGemm* dense_down = nullptr) {
   const int P = T * d->k;
   const int NC = (P + kPairChunk - 1) / kPairChunk;
   if (sorted) {
@@ -315,8 +316,10 @@ static moe_status run_routed(const moe_desc* d, const void* x, int32_t T, const 
   if (path == MOE_PATH_GEMM) {
     MOE_LAUNCH("gather_rows", stream, launch_gather_rows(*d, x, ws, P, dev->num_sms, stream));
     const int chunk = chunk_tokens(T, d->k, d->E);
-    MOE_LAUNCH("gemm_gateup", stream, launch_gemm_gateup(*d, ws, P, chunk, dev->num_sms, dev->flags, stream));
-    MOE_LAUNCH("gemm_down", stream, launch_gemm_down(*d, topk_w, ws, P, chunk, dev->num_sms, dev->flags, stream));
+    MOE_LAUNCH("gemm_gateup", stream,
+               launch_gemm_gateup(*d, ws, P, chunk, dev->num_sms, dev->flags, stream, dense_up));
+    MOE_LAUNCH("gemm_down", stream,
+               launch_gemm_down(*d, topk_w, ws, P, chunk, dev->num_sms, dev->flags, stream, dense_down));
   } else {
     MOE_LAUNCH("gemv_gateup", stream, launch_gemv_gateup(*d, x, d->k, ws, dev->num_sms, dev->flags, stream));
     MOE_LAUNCH("gemv_down", stream, launch_gemv_down(*d, topk_w, d->k, ws, dev->num_sms, dev->flags, stream));
@@ -473,8 +476,18 @@ extern "C" moe_status moe_forward_block(const moe_desc* d, const moe_shared_expe
   DeviceState* dev = nullptr;
   if ((st = device_state(&dev)) != MOE_OK) return st;
   const Workspace ws = carve_workspace(*d, T, workspace);
-  if ((st = run_routed(d, x, T, topk_idx, topk_w, ws, path, dev, stream)) != MOE_OK) return st;
   const float* ys = nullptr;
+  if (shared && path == MOE_PATH_GEMM && spath == MOE_PATH_GEMM && sd.wfmt == d->wfmt) {
+    // the shared expert's units ride in the routed experts' grouped-GEMM launches
+    const Workspace ss = carve_workspace(sd, T, static_cast<char*>(workspace) + shared_off);
+    const int chunk = chunk_tokens(T, sd.k, sd.E);
+    const DenseGemm up{&sd, x, ss.hbuf, T, chunk};
+    const DenseGemm down{&sd, ss.hbuf, ss.yp, T, chunk};
+    if ((st = run_routed(d, x, T, topk_idx, topk_w, ws, path, dev, stream, false, &up, &down)) != MOE_OK) return st;
+    MOE_LAUNCH("combine", stream, launch_combine(*d, topk_idx, T, ws.yp, y, stream, ss.yp, residual));
+    return MOE_OK;
+  }
+  if ((st = run_routed(d, x, T, topk_idx, topk_w, ws, path, dev, stream)) != MOE_OK) return st;
   if (shared) {
     Workspace ss = carve_workspace(sd, T, static_cast<char*>(workspace) + shared_off);
     float* ones = reinterpret_cast<float*>(static_cast<char*>(workspace) + ones_off);
