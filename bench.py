@@ -292,8 +292,10 @@ def run_reference(args):
     t0 = time.perf_counter()
     oracle_step(orc, [0])
     per_token = max(time.perf_counter() - t0, 1e-6)
-    # each step: a token sample worth about 6 s of oracle work on all cores
-    n = max(1, min(prob.T, int(6.0 * cores / per_token)))
+    # each step: a token sample sized so that the whole run (warm-up + timed steps) is
+    # about two minutes of oracle work on all cores, at most 6 s per step
+    per_step_s = min(6.0, 120.0 / max(1, args.steps + args.warmup))
+    n = max(1, min(prob.T, int(per_step_s * cores / per_token)))
     rng = np.random.default_rng(1)
     times = []
     for step in range(args.warmup + args.steps):
