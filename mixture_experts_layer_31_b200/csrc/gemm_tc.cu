@@ -32,6 +32,12 @@
 // TMEM holds two accumulator buffers when they fit (chunks up to 128 tokens),
 // so the epilogue of one unit overlaps the MMAs of the next.  Every wait is
 // bounded (MOE_FLAG_TIMEOUT).
+// A launch may carry a second, dense problem (the shared expert of the MoE
+// block: every token in order, weight 1, weights of its own) whose units follow
+// the routed ones, so both share the persistent grid.
+// The router's logits reuse the kernel as a third mode (MODE 2): dense
+// x . W3^T over K splits, W3 the exact three-way bf16 split of the fp32 router
+// weights.
 // No cluster, no multicast.
 #include <cuda.h>
 
