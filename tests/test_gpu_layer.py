@@ -88,3 +88,44 @@ def test_layer_forward_launches_fewer_kernels_at_decode():
     layer(x)
     separate = moe.moe_launch_count() - n0
     assert fused == separate - 1  # top-k and sort share one launch
+
+
+EDGE = {
+    "max-H-decode": (2, dict(T=32, H=8192, E=16, I=64)),       # decode logits split 8 ways (213 KB of smem)
+    "max-I-decode": (2, dict(T=8, H=256, E=8, I=8192)),
+    "k1-decode": (3, dict(T=17, H=256, E=24, I=128, k=1)),
+    "k-equals-active": (5, dict(T=12, H=256, E=32, I=128, n_active=8, bias=("skew", 0.1))),
+    "fp32-H64": (1, dict(T=5, H=64, E=8, k=2, I=64)),
+}
+
+
+@pytest.mark.parametrize("name", list(EDGE))
+def test_layer_forward_edge_shapes(name):
+    cid, over = EDGE[name]
+    prob = synth.make_problem(cid, **over)
+    layer = layer_from_problem(prob)
+    y, idx, w = layer.layer(x_to_device(prob))
+    torch.cuda.synchronize()
+    judge(prob, y, idx, w)
+    if prob.mask is not None:
+        assert prob.mask[idx.cpu().numpy()].all()
+
+
+def test_zero_tokens_is_a_no_op_on_every_entry_point():
+    prob = synth.make_problem(2, T=4, H=256, E=16, I=128, shared=128, residual=True)
+    layer = layer_from_problem(prob)
+    x = x_to_device(prob)[:0]
+    idx = torch.empty((0, prob.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((0, prob.k), dtype=torch.float32, device="cuda")
+    y = torch.empty((0, prob.H), dtype=torch.bfloat16, device="cuda")
+    n0 = moe.moe_launch_count()
+    ws = layer.workspace(1)
+    moe.moe_layer_forward(layer.desc, x.data_ptr() or 256, 0, idx.data_ptr() or 256, w.data_ptr() or 256,
+                          y.data_ptr() or 256, ws.data_ptr(), ws.numel())
+    moe.moe_forward_block(layer.desc, layer.shared, x.data_ptr() or 256, 0, idx.data_ptr() or 256,
+                          w.data_ptr() or 256, None, y.data_ptr() or 256, ws.data_ptr(), ws.numel())
+    counts = torch.zeros(prob.E, dtype=torch.uint64, device="cuda")
+    moe.moe_expert_counts(layer.desc, idx.data_ptr() or 256, 0, counts.data_ptr())
+    torch.cuda.synchronize()
+    assert moe.moe_launch_count() == n0
+    assert int(counts.sum()) == 0
