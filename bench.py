@@ -149,6 +149,25 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def gpu_context(gpu_index: int) -> dict:
+    """Driver version and the compute processes visible on the GPU other than this
+    one (a run that shared its GPU is not a clean number)."""
+    out = {"driver": None, "other_processes": None}
+    try:
+        r = subprocess.run(["nvidia-smi", "-i", str(gpu_index), "--query-gpu=driver_version,uuid",
+                            "--format=csv,noheader"], capture_output=True, text=True, timeout=20)
+        drv, uuid = [c.strip() for c in r.stdout.strip().splitlines()[0].split(",")][:2]
+        out["driver"] = drv
+        r = subprocess.run(["nvidia-smi", "--query-compute-apps=gpu_uuid,pid", "--format=csv,noheader"],
+                           capture_output=True, text=True, timeout=20)
+        pids = [l.split(",")[1].strip() for l in r.stdout.strip().splitlines()
+                if "," in l and l.split(",")[0].strip() == uuid]
+        out["other_processes"] = len([p for p in pids if p != str(os.getpid())])
+    except (OSError, subprocess.SubprocessError, IndexError, ValueError):
+        pass
+    return out
+
+
 # ----------------------------------------------------------------------------- workload accounting
 
 def touched_experts(idx: np.ndarray, E: int) -> int:
@@ -472,7 +491,8 @@ def run_ours(args):
                                           + (0 if res is None else int(res.numel() * res.element_size())),
                     "d2h_bytes_per_step": int(y.numel() * y.element_size())},
             "gpu_launches": int(launches),
-            "clocks": clocks.summary()}
+            "clocks": clocks.summary(),
+            "gpu": gpu_context(local)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample = time_oracle(prob, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}

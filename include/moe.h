@@ -261,6 +261,16 @@ MOE_API moe_status moe_expert_counts(const moe_desc* d, const int32_t* topk_idx,
 MOE_API moe_status moe_cover_set(const uint64_t* counts, int32_t E, double cover, uint8_t* keep,
                                  int32_t* new_index, int32_t* n_keep);
 
+/*
+ * Diagnostic (the pages have no counterpart): launches one small kernel whose
+ * only waiting thread waits on a barrier that nothing completes.  After the
+ * library's in-kernel wait bound (2 s of GPU time) it gives up, raises
+ * MOE_FLAG_TIMEOUT in the device flags and returns; the context stays usable.
+ * Shows on a given device that the library's waits end by themselves.
+ * Asynchronous; read the result with moe_device_flags().
+ */
+MOE_API moe_status moe_selftest_bounded_wait(cudaStream_t stream);
+
 /* Message for the last non-OK status returned on this thread ("" if none). */
 MOE_API const char* moe_last_error(void);
 

@@ -39,8 +39,8 @@ ROUTER = {"sigmoid": MOE_ROUTER_SIGMOID_BIAS, "softmax": MOE_ROUTER_SOFTMAX}
 EXPORTS = ("moe_workspace_size", "moe_route", "moe_forward", "moe_layer_forward", "moe_forward_noalloc",
            "moe_block_workspace_size",
            "moe_forward_block", "moe_expert_counts",
-           "moe_cover_set", "moe_last_error", "moe_device_flags", "moe_launch_count", "moe_stage_timing",
-           "moe_stage_times")
+           "moe_cover_set", "moe_selftest_bounded_wait", "moe_last_error", "moe_device_flags", "moe_launch_count",
+           "moe_stage_timing", "moe_stage_times")
 MOE_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -88,6 +88,8 @@ def _load() -> ctypes.CDLL:
     lib.moe_forward_block.argtypes = [D, SH, vp, i32, vp, vp, vp, vp, vp, sz, vp]
     lib.moe_expert_counts.argtypes = [D, vp, i32, vp, vp]
     lib.moe_cover_set.argtypes = [vp, i32, ctypes.c_double, vp, vp, ctypes.POINTER(i32)]
+    lib.moe_selftest_bounded_wait.argtypes = [vp]
+    lib.moe_selftest_bounded_wait.restype = ctypes.c_int
     lib.moe_last_error.argtypes = []
     lib.moe_last_error.restype = ctypes.c_char_p
     lib.moe_device_flags.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
@@ -183,6 +185,11 @@ def moe_cover_set(counts, cover: float):
     _check(lib().moe_cover_set(c.ctypes.data, int(E), float(cover), keep.ctypes.data, new_index.ctypes.data,
                                ctypes.byref(n)))
     return keep, new_index, int(n.value)
+
+
+def moe_selftest_bounded_wait(stream: int = 0) -> None:
+    """Launch the bounded-wait self-test (raises MOE_FLAG_TIMEOUT on the device after ~2 s)."""
+    _check(lib().moe_selftest_bounded_wait(stream))
 
 
 def moe_last_error() -> str:

@@ -14,6 +14,9 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
+#include "common.cuh"
 #include "internal.h"
 #include "moe.h"
 
@@ -93,8 +96,10 @@ static cudaEvent_t pool_event() {
   return ev;
 }
 
+// every launch sits in an NVTX range named after the kernel's stage (visible to
+// profilers; a no-op without one attached)
 void* launch_start(const char* name, cudaStream_t s) {
-  (void)name;
+  nvtxRangePushA(name);
   if (!g_timing.load(std::memory_order_relaxed)) return nullptr;
   std::lock_guard<std::mutex> lk(g_time_mu);
   cudaEvent_t ev = pool_event();
@@ -104,6 +109,7 @@ void* launch_start(const char* name, cudaStream_t s) {
 
 cudaError_t launch_done(const char* name, cudaStream_t s, void* begin_event) {
   cudaError_t err = cudaGetLastError();
+  nvtxRangePop();
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (begin_event) {
     std::lock_guard<std::mutex> lk(g_time_mu);
@@ -551,6 +557,33 @@ extern "C" moe_status moe_cover_set(const uint64_t* counts, int32_t E, double co
   int32_t next = 0;
   for (int32_t e = 0; e < E; ++e) new_index[e] = keep[e] ? next++ : -1;
   *n_keep = m;
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------------ diagnostics
+
+namespace moe {
+namespace {
+// one thread waits on an mbarrier that nothing completes: the library's bounded
+// wait gives up, the kernel raises MOE_FLAG_TIMEOUT and returns
+__global__ void bounded_wait_selftest_kernel(uint32_t* flags) {
+  __shared__ __align__(8) uint64_t never;
+  if (threadIdx.x == 0) {
+    mbar_init(&never, 1);
+    fence_mbar_init();
+    if (!mbar_wait(&never, 0)) raise_flag(flags, MOE_FLAG_TIMEOUT);
+  }
+}
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status moe_selftest_bounded_wait(cudaStream_t stream) {
+  g_err.clear();
+  DeviceState* dev = nullptr;
+  moe_status st = device_state(&dev);
+  if (st != MOE_OK) return st;
+  MOE_LAUNCH("selftest_bounded_wait", stream, launch_k(bounded_wait_selftest_kernel, dim3(1), dim3(32), 0, stream,
+                                                        dev->flags));
   return MOE_OK;
 }
 
