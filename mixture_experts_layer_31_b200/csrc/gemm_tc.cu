@@ -54,6 +54,7 @@ constexpr int kBoxRows = 32;               // token rows per TMA box
 constexpr int kMaxStages = 16;
 constexpr int kAStages = 2;                // quantised: bf16 A tiles between dequant and MMA
 constexpr int kBarrierBytes = 1024;
+constexpr int kUnitQ = 8;                  // expert GEMMs: unit ids in flight between the scheduler and the roles
 constexpr int kSmemLimit = 232448;         // 227 KB opt-in
 
 struct GemmArgs {
@@ -93,6 +94,10 @@ struct GemmArgs {
   const float* sd0;
   const float* sd1;
   void* outd;           // gate/up: h [Td, Rd] bf16; down: rows [Td, Rd] fp32
+  // expert GEMMs: units past the first one of each CTA are claimed from this
+  // counter (zeroed by the kernel that runs before the launch), so CTAs whose
+  // units are cheap take more of them
+  int* sched;
 };
 
 __device__ __forceinline__ void wait_or_die(uint64_t* bar, uint32_t parity, bool& dead, uint32_t* flags) {
@@ -254,7 +259,10 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
   uint64_t* acc_full = a_empty + kAStages;             // [2]
   uint64_t* acc_empty = acc_full + 2;                  // [2]
   uint64_t* mma_done = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* q_full = mma_done + 1;                     // [kUnitQ] unit id published
+  uint64_t* q_empty = q_full + kUnitQ;                 // [kUnitQ] every role has read it
+  int* unit_q = reinterpret_cast<int*>(q_empty + kUnitQ);  // [kUnitQ]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unit_q + kUnitQ);
   float* xchg = reinterpret_cast<float*>(smem + kBarrierBytes);
   uint8_t* a_ring = smem + kBarrierBytes + Tr::kXchg;  // quantised: kAStages x MT bf16 A tiles
   uint8_t* stages = a_ring + (Tr::kQuant ? kAStages * MT * kTileBytes : 0);
@@ -281,6 +289,12 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
       mbar_init(&acc_empty[i], Tr::kEpiWarps);
     }
     mbar_init(mma_done, 1);
+    // readers of a queue slot: the MMA warp, the epilogue warps and, for quantised
+    // weights, the token producer and the dequant warps
+    for (int i = 0; i < kUnitQ; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1 + Tr::kEpiWarps + (Tr::kQuant ? 1 + Tr::kDequantWarps : 0));
+    }
     fence_mbar_init();
   }
   if (w == 1) tmem_alloc(tmem_slot, (uint32_t)a.tmem_cols);
@@ -305,6 +319,36 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
                                : (ntouched > 0 ? a.meta[3] * nib : 0);
   const int total = routed + (MODE == 2 ? 0 : a.dense_units);
 
+  // The sequence of units of this CTA.  Router (uniform units): blockIdx.x + i *
+  // gridDim.x.  Expert GEMMs: the first unit is blockIdx.x, each later one is
+  // claimed from a.sched by warp 0 lane 0 when it starts loading it, and
+  // published through a small queue that every other role reads in order; -1
+  // ends the sequence.
+  auto publish_unit = [&](uint32_t i, bool& dead) -> int {
+    if (MODE == 2) {
+      const int u = blockIdx.x + (int)i * gridDim.x;
+      return u < total ? u : -1;
+    }
+    const int slot = i % kUnitQ;
+    wait_or_die(&q_empty[slot], ((i / kUnitQ) & 1u) ^ 1u, dead, a.flags);
+    int u = i == 0 ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(a.sched, 1);
+    if (u >= total || dead) u = -1;
+    unit_q[slot] = u;
+    mbar_arrive(&q_full[slot]);  // release: readers that see the phase see the id
+    return u;
+  };
+  auto read_unit = [&](uint32_t i, bool& dead) -> int {  // one lane per reading warp
+    if (MODE == 2) {
+      const int u = blockIdx.x + (int)i * gridDim.x;
+      return u < total ? u : -1;
+    }
+    const int slot = i % kUnitQ;
+    wait_or_die(&q_full[slot], (i / kUnitQ) & 1u, dead, a.flags);
+    const int u = dead ? -1 : unit_q[slot];
+    mbar_arrive(&q_empty[slot]);
+    return u;
+  };
+
   if (w == 0 || (Tr::kQuant && w == 2)) {
     // ------------------------------------------------------------------ TMA producers
     // bf16: warp 0 loads A and B into one stage.  Quantised: warp 0 loads the raw
@@ -318,7 +362,9 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
       bool dead = false;
       uint32_t it = 0;
       const uint32_t abytes = load_a ? MT * (Tr::kQuant ? Tr::kRawTile : kTileBytes) : 0;
-      for (int u = blockIdx.x; u < total; u += gridDim.x) {
+      for (uint32_t i = 0;; ++i) {
+        const int u = w == 0 ? publish_unit(i, dead) : read_unit(i, dead);
+        if (u < 0) break;
         const Unit t = decode_unit<MODE>(a, u, nib, ntouched, routed);
         const int nbox = load_b ? (t.n_tok + kBoxRows - 1) / kBoxRows : 0;
         const int brow = t.pos0;
@@ -359,10 +405,12 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool dead = false;
-      uint32_t it = 0, local = 0;
+      uint32_t it = 0;
       const uint32_t stage0 = smem_u32(stages);
       const uint32_t a_ring0 = smem_u32(a_ring);
-      for (int u = blockIdx.x; u < total; u += gridDim.x, ++local) {
+      for (uint32_t local = 0;; ++local) {
+        const int u = read_unit(local, dead);
+        if (u < 0) break;
         const Unit t = decode_unit<MODE>(a, u, nib, ntouched, routed);
         const uint32_t buf = local % nbuf;
         wait_or_die(&acc_empty[buf], ((local / nbuf) & 1u) ^ 1u, dead, a.flags);
@@ -407,8 +455,11 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
     const int bar_x = 1 + 2 * grp, bar_v = 2 + 2 * grp;
     float* gx = xchg + grp * (Tr::kGroupXchg / 4);
     bool dead = false;
-    uint32_t local = 0;
-    for (int u = blockIdx.x; u < total; u += gridDim.x, ++local) {
+    for (uint32_t local = 0;; ++local) {
+      int u = 0;
+      if (lane == 0) u = read_unit(local, dead);
+      u = __shfl_sync(0xFFFFFFFFu, u, 0);
+      if (u < 0) break;
       const Unit t = decode_unit<MODE>(a, u, nib, ntouched, routed);
       const uint32_t buf = local % nbuf;
       if (lane == 0) wait_or_die(&acc_full[buf], (local / nbuf) & 1u, dead, a.flags);
@@ -504,7 +555,11 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
     const int c8 = ct & 7, r0 = ct >> 3;
     bool dead = false;
     uint32_t it = 0;
-    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+    for (uint32_t i = 0;; ++i) {
+      int u = 0;
+      if (lane == 0) u = read_unit(i, dead);
+      u = __shfl_sync(0xFFFFFFFFu, u, 0);
+      if (u < 0) break;
       const Unit t = decode_unit<MODE>(a, u, nib, ntouched, routed);
       // int4: block scales of this thread's rows, one K step ahead
       const ProbView pv = view_of(a, t);
@@ -695,9 +750,14 @@ GemmArgs common(const Workspace& ws, int chunk, uint32_t* flags) {
   return a;
 }
 
+// also zeroes the unit counters of the two expert GEMMs that follow (meta[8], meta[9])
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x, int H, int k,
                                                           const int32_t* __restrict__ sorted_pair,
-                                                          const int32_t* __restrict__ meta, uint16_t* __restrict__ xs) {
+                                                          int32_t* __restrict__ meta, uint16_t* __restrict__ xs) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    meta[8] = 0;
+    meta[9] = 0;
+  }
   const int P = meta[1];
   const int per_row = H / 8;  // 16-byte chunks
   const size_t n = (size_t)P * per_row;
@@ -798,8 +858,7 @@ cudaError_t launch_gather_rows(const moe_desc& d, const void* x, const Workspace
   if (blocks > num_sms * 8) blocks = num_sms * 8;
   if (blocks < 1) blocks = 1;
   return launch_k(gather_rows_kernel, dim3(blocks), dim3(256), 0, s, static_cast<const uint16_t*>(x), d.H, d.k,
-                    static_cast<const int32_t*>(ws.sorted_pair), static_cast<const int32_t*>(ws.meta),
-                    static_cast<uint16_t*>(ws.xs));
+                    static_cast<const int32_t*>(ws.sorted_pair), ws.meta, static_cast<uint16_t*>(ws.xs));
 }
 
 cudaError_t launch_gemm_gateup(const moe_desc& d, const Workspace& ws, int P, int chunk, int num_sms,
@@ -819,6 +878,7 @@ cudaError_t launch_gemm_gateup(const moe_desc& d, const Workspace& ws, int P, in
   a.K = d.H;
   a.act = d.act;
   a.qsh = d.wfmt == MOE_W_INT4_B128 ? 7 : 5;
+  a.sched = ws.meta + 8;
   m.w0d = m.w0;
   m.w1d = m.w1;
   m.bd = m.b;
@@ -856,6 +916,7 @@ cudaError_t launch_gemm_down(const moe_desc& d, const float* topk_w, const Works
   a.R = d.H;
   a.K = d.I;
   a.qsh = d.wfmt == MOE_W_INT4_B128 ? 7 : 5;
+  a.sched = ws.meta + 9;
   m.w1 = m.w0;
   m.w0d = m.w0;
   m.w1d = m.w0;

@@ -51,7 +51,7 @@ struct Workspace {
   int32_t* offsets;   // [E + 1] start of each expert in the sorted order
   int32_t* touched;   // [E] experts with count > 0, ascending; touched[E] unused
   int32_t* meta;      // [16] device scalars: [0] touched experts, [1] valid pairs, [2] token groups,
-                      //       [3] token chunks
+                      //       [3] token chunks, [8] / [9] unit counters of the gate/up and down GEMMs
   int32_t* group_base;  // [E + 1] first token group of each touched expert (touched order)
   int32_t* tile_base;   // [E + 1] first token chunk of each touched expert
   int32_t* sorted_pair;  // [P] pair id (t * k + slot) at each sorted position

@@ -179,6 +179,8 @@ __global__ void __launch_bounds__(256) dense_plan_kernel(int T, int chunk, int32
     meta[1] = T;
     meta[2] = groups;
     meta[3] = chunks;
+    meta[8] = 0;  // unit counters of the expert GEMMs that follow
+    meta[9] = 0;
   }
 }
 
