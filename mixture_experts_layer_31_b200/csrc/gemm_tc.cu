@@ -482,20 +482,33 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
           const size_t grow = (size_t)t.e * pv.R + (live ? row : 0);
           const float sg = WF == MOE_W_INT8_ROW ? pv.s0[grow] : 1.f;
           const float su = WF == MOE_W_INT8_ROW ? pv.s1[grow] : 1.f;
-          uint16_t* hout = static_cast<uint16_t*>(pv.out);
+          uint16_t* hout = static_cast<uint16_t*>(pv.out) + (size_t)pos0 * pv.R + row;
+          const bool gelu = a.act == MOE_ACT_GELU_TANH;
           for (int n0 = c_first; n0 < t.n_tok; n0 += c_step) {
             uint32_t g[16], v[16];
             tmem_ld16(tacc + n0, g);
             tmem_ld16(tacc + a.acc_stride + n0, v);
             tmem_ld_wait();
             if (live) {
+              // all 16 values first (independent chains), then the stores
+              uint16_t hv[16];
+              if (gelu) {
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                if (n0 + j < t.n_tok) {
-                  const float gv = __uint_as_float(g[j]) * sg, uv = __uint_as_float(v[j]) * su;
-                  const float hv = a.act == MOE_ACT_GELU_TANH ? gelu_tanh_mul_fast(gv, uv) : silu_mul_fast(gv, uv);
-                  hout[(size_t)(pos0 + n0 + j) * pv.R + row] = f32_to_bf16(hv);
-                }
+                for (int j = 0; j < 16; ++j)
+                  hv[j] = f32_to_bf16(gelu_tanh_mul_fast(__uint_as_float(g[j]) * sg, __uint_as_float(v[j]) * su));
+              } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                  hv[j] = f32_to_bf16(silu_mul_fast(__uint_as_float(g[j]) * sg, __uint_as_float(v[j]) * su));
+              }
+              uint16_t* dst = hout + (size_t)n0 * pv.R;
+              if (n0 + 16 <= t.n_tok) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) dst[(size_t)j * pv.R] = hv[j];
+              } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                  if (n0 + j < t.n_tok) dst[(size_t)j * pv.R] = hv[j];
               }
             }
           }
@@ -532,10 +545,25 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
             uint32_t v[16];
             tmem_ld16(tacc + n0, v);
             tmem_ld_wait();
+            if (n0 + 16 <= t.n_tok) {
+              // whole chunk: pair ids and weights as 16-byte broadcasts, stores unpredicated
+              const int4* p4 = reinterpret_cast<const int4*>(s_pair + n0);
+              const float4* w4 = reinterpret_cast<const float4*>(s_w + n0);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              if (n0 + j < t.n_tok)
-                yp[(size_t)s_pair[n0 + j] * pv.R + row] = s_w[n0 + j] * sd * __uint_as_float(v[j]);
+              for (int j4 = 0; j4 < 4; ++j4) {
+                const int4 p = p4[j4];
+                const float4 wv = w4[j4];
+                yp[(size_t)p.x * pv.R + row] = wv.x * sd * __uint_as_float(v[4 * j4 + 0]);
+                yp[(size_t)p.y * pv.R + row] = wv.y * sd * __uint_as_float(v[4 * j4 + 1]);
+                yp[(size_t)p.z * pv.R + row] = wv.z * sd * __uint_as_float(v[4 * j4 + 2]);
+                yp[(size_t)p.w * pv.R + row] = wv.w * sd * __uint_as_float(v[4 * j4 + 3]);
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                if (n0 + j < t.n_tok)
+                  yp[(size_t)s_pair[n0 + j] * pv.R + row] = s_w[n0 + j] * sd * __uint_as_float(v[j]);
+              }
             }
           }
         }
