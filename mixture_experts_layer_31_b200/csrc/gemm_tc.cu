@@ -53,7 +53,7 @@ constexpr int kTileBytes = kBM * kBK * 2;  // A tile, 16 KB
 constexpr int kBoxRows = 32;               // token rows per TMA box
 constexpr int kMaxStages = 16;
 constexpr int kAStages = 2;                // quantised: bf16 A tiles between dequant and MMA
-constexpr int kBarrierBytes = 1024;
+constexpr int kBarrierBytes = 2048;          // barriers, the unit queue, the TMEM address
 constexpr int kUnitQ = 8;                  // expert GEMMs: unit ids in flight between the scheduler and the roles
 constexpr int kSmemLimit = 232448;         // 227 KB opt-in
 
@@ -114,6 +114,12 @@ struct Unit {
   int pos0;    // first sorted position (dense: first token) of the unit's chunk
   bool dense;  // a unit of the dense problem
 };
+
+// barriers [4 rings x kMaxStages, 2 x kAStages, acc_full/acc_empty x 2, mma_done,
+// q_full/q_empty x kUnitQ], the unit queue (ids and decoded units), the TMEM address
+static_assert((4 * kMaxStages + 2 * kAStages + 5 + 2 * kUnitQ) * 8 + kUnitQ * (4 + (int)sizeof(Unit)) + 4 <=
+                  kBarrierBytes,
+              "barrier region too small");
 
 // The per-problem view a role needs for a unit.
 struct ProbView {
@@ -183,6 +189,20 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u, int nib, i
   t.nk = nk_all;
   t.pos0 = t.base + t.c * a.chunk;
   return t;
+}
+
+// lane 0's unit to the whole warp
+__device__ __forceinline__ void shfl_unit(Unit& t) {
+  t.e = __shfl_sync(0xFFFFFFFFu, t.e, 0);
+  t.base = __shfl_sync(0xFFFFFFFFu, t.base, 0);
+  t.ib = __shfl_sync(0xFFFFFFFFu, t.ib, 0);
+  t.c = __shfl_sync(0xFFFFFFFFu, t.c, 0);
+  t.n_tok = __shfl_sync(0xFFFFFFFFu, t.n_tok, 0);
+  t.n_mma = __shfl_sync(0xFFFFFFFFu, t.n_mma, 0);
+  t.k0 = __shfl_sync(0xFFFFFFFFu, t.k0, 0);
+  t.nk = __shfl_sync(0xFFFFFFFFu, t.nk, 0);
+  t.pos0 = __shfl_sync(0xFFFFFFFFu, t.pos0, 0);
+  t.dense = __shfl_sync(0xFFFFFFFFu, t.dense ? 1 : 0, 0) != 0;
 }
 
 // Raw bytes of one 8-element chunk: 8 bytes of int8, or 4 bytes of packed int4
@@ -261,8 +281,9 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
   uint64_t* mma_done = acc_empty + 2;
   uint64_t* q_full = mma_done + 1;                     // [kUnitQ] unit id published
   uint64_t* q_empty = q_full + kUnitQ;                 // [kUnitQ] every role has read it
-  int* unit_q = reinterpret_cast<int*>(q_empty + kUnitQ);  // [kUnitQ]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unit_q + kUnitQ);
+  int* unit_q = reinterpret_cast<int*>(q_empty + kUnitQ);  // [kUnitQ] unit ids
+  Unit* unit_tq = reinterpret_cast<Unit*>(unit_q + kUnitQ);  // [kUnitQ] the same units, decoded
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unit_tq + kUnitQ);
   float* xchg = reinterpret_cast<float*>(smem + kBarrierBytes);
   uint8_t* a_ring = smem + kBarrierBytes + Tr::kXchg;  // quantised: kAStages x MT bf16 A tiles
   uint8_t* stages = a_ring + (Tr::kQuant ? kAStages * MT * kTileBytes : 0);
@@ -324,27 +345,36 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
   // claimed from a.sched by warp 0 lane 0 when it starts loading it, and
   // published through a small queue that every other role reads in order; -1
   // ends the sequence.
-  auto publish_unit = [&](uint32_t i, bool& dead) -> int {
+  // The scheduler decodes each unit once (a binary search over global memory)
+  // and publishes it decoded, so the other roles read it from shared memory.
+  auto publish_unit = [&](uint32_t i, bool& dead, Unit& t) -> int {
     if (MODE == 2) {
       const int u = blockIdx.x + (int)i * gridDim.x;
+      if (u < total) t = decode_unit<MODE>(a, u, nib, ntouched, routed);
       return u < total ? u : -1;
     }
     const int slot = i % kUnitQ;
     wait_or_die(&q_empty[slot], ((i / kUnitQ) & 1u) ^ 1u, dead, a.flags);
     int u = i == 0 ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(a.sched, 1);
     if (u >= total || dead) u = -1;
+    if (u >= 0) {
+      t = decode_unit<MODE>(a, u, nib, ntouched, routed);
+      unit_tq[slot] = t;
+    }
     unit_q[slot] = u;
-    mbar_arrive(&q_full[slot]);  // release: readers that see the phase see the id
+    mbar_arrive(&q_full[slot]);  // release: readers that see the phase see the id and the unit
     return u;
   };
-  auto read_unit = [&](uint32_t i, bool& dead) -> int {  // one lane per reading warp
+  auto read_unit = [&](uint32_t i, bool& dead, Unit& t) -> int {  // one lane per reading warp
     if (MODE == 2) {
       const int u = blockIdx.x + (int)i * gridDim.x;
+      if (u < total) t = decode_unit<MODE>(a, u, nib, ntouched, routed);
       return u < total ? u : -1;
     }
     const int slot = i % kUnitQ;
     wait_or_die(&q_full[slot], (i / kUnitQ) & 1u, dead, a.flags);
     const int u = dead ? -1 : unit_q[slot];
+    if (u >= 0) t = unit_tq[slot];
     mbar_arrive(&q_empty[slot]);
     return u;
   };
@@ -361,11 +391,13 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
       uint64_t* re = raw ? rempty : empty;
       bool dead = false;
       uint32_t it = 0;
+      int rs = 0;        // ring slot of K step `it`
+      uint32_t rph = 0;  // and its phase parity
       const uint32_t abytes = load_a ? MT * (Tr::kQuant ? Tr::kRawTile : kTileBytes) : 0;
       for (uint32_t i = 0;; ++i) {
-        const int u = w == 0 ? publish_unit(i, dead) : read_unit(i, dead);
+        Unit t{};
+        const int u = w == 0 ? publish_unit(i, dead, t) : read_unit(i, dead, t);
         if (u < 0) break;
-        const Unit t = decode_unit<MODE>(a, u, nib, ntouched, routed);
         const int nbox = load_b ? (t.n_tok + kBoxRows - 1) / kBoxRows : 0;
         const int brow = t.pos0;
         const int wrow0 = t.e * (t.dense ? a.Rd : a.R) + t.ib * Tr::kRows;
@@ -373,8 +405,10 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
         const CUtensorMap* mw1 = t.dense ? &tm_w1d : &tm_w1;
         const CUtensorMap* mb = t.dense ? &tm_bd : &tm_b;
         for (int kb = t.k0; kb < t.k0 + t.nk; ++kb, ++it) {
-          const int s = it % ring;
-          wait_or_die(&re[s], ((it / ring) & 1u) ^ 1u, dead, a.flags);
+          const int s = rs;
+          const uint32_t ph = rph;
+          if (++rs == ring) { rs = 0; rph ^= 1u; }
+          wait_or_die(&re[s], ph ^ 1u, dead, a.flags);
           if (dead) continue;
           mbar_arrive_expect_tx(&rf[s], abytes + nbox * kBoxRows * kBK * 2);
           if (load_a) {
@@ -406,22 +440,26 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
     if (lane == 0) {
       bool dead = false;
       uint32_t it = 0;
+      int ms = 0;        // main-ring slot of K step `it`
+      uint32_t mph = 0;  // and its phase parity
       const uint32_t stage0 = smem_u32(stages);
       const uint32_t a_ring0 = smem_u32(a_ring);
       for (uint32_t local = 0;; ++local) {
-        const int u = read_unit(local, dead);
+        Unit t{};
+        const int u = read_unit(local, dead, t);
         if (u < 0) break;
-        const Unit t = decode_unit<MODE>(a, u, nib, ntouched, routed);
         const uint32_t buf = local % nbuf;
         wait_or_die(&acc_empty[buf], ((local / nbuf) & 1u) ^ 1u, dead, a.flags);
         tc_fence_after();
         const uint32_t idesc = umma_idesc_bf16(kBM, t.n_mma);
         const uint32_t d = tmem_base + buf * buf_cols;
         for (int kb = 0; kb < t.nk; ++kb, ++it) {
-          const int s = it % NS;
+          const int s = ms;
+          const uint32_t ph = mph;
+          if (++ms == NS) { ms = 0; mph ^= 1u; }
           const int ja = it % kAStages;
           if (Tr::kQuant) wait_or_die(&ready[ja], (it / kAStages) & 1u, dead, a.flags);
-          wait_or_die(&full[s], (it / NS) & 1u, dead, a.flags);
+          wait_or_die(&full[s], ph, dead, a.flags);
           if (dead) continue;
           tc_fence_after();
           const uint32_t sb = stage0 + s * a.stage_bytes;
@@ -457,10 +495,11 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
     bool dead = false;
     for (uint32_t local = 0;; ++local) {
       int u = 0;
-      if (lane == 0) u = read_unit(local, dead);
+      Unit t{};
+      if (lane == 0) u = read_unit(local, dead, t);
       u = __shfl_sync(0xFFFFFFFFu, u, 0);
       if (u < 0) break;
-      const Unit t = decode_unit<MODE>(a, u, nib, ntouched, routed);
+      shfl_unit(t);
       const uint32_t buf = local % nbuf;
       if (lane == 0) wait_or_die(&acc_full[buf], (local / nbuf) & 1u, dead, a.flags);
       if (MODE != 1) {
@@ -583,12 +622,15 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
     const int c8 = ct & 7, r0 = ct >> 3;
     bool dead = false;
     uint32_t it = 0;
+    int rs = 0;        // raw-ring slot of K step `it`
+    uint32_t rph = 0;  // and its phase parity
     for (uint32_t i = 0;; ++i) {
       int u = 0;
-      if (lane == 0) u = read_unit(i, dead);
+      Unit t{};
+      if (lane == 0) u = read_unit(i, dead, t);
       u = __shfl_sync(0xFFFFFFFFu, u, 0);
       if (u < 0) break;
-      const Unit t = decode_unit<MODE>(a, u, nib, ntouched, routed);
+      shfl_unit(t);
       // int4: block scales of this thread's rows, one K step ahead
       const ProbView pv = view_of(a, t);
       const float* srow[kPer];
@@ -611,9 +653,11 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
           if (WF == MOE_W_INT4_B32 && kb + 1 < t.nk)
             sc_next[j] = __ldg(srow[j] + (((t.k0 + kb + 1) * kBK + c8 * 8) >> a.qsh));
         }
-        const int s = it % a.RS;
+        const int s = rs;
+        const uint32_t ph = rph;
+        if (++rs == a.RS) { rs = 0; rph ^= 1u; }
         const int ja = it % kAStages;
-        wait_or_die(&rfull[s], (it / a.RS) & 1u, dead, a.flags);
+        wait_or_die(&rfull[s], ph, dead, a.flags);
         wait_or_die(&a_empty[ja], ((it / kAStages) & 1u) ^ 1u, dead, a.flags);
         if (!dead) {
           const uint8_t* raw = raw_ring + (size_t)s * a.raw_stage_bytes;
