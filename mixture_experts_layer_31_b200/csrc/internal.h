@@ -51,7 +51,8 @@ struct Workspace {
   int32_t* offsets;   // [E + 1] start of each expert in the sorted order
   int32_t* touched;   // [E] experts with count > 0, ascending; touched[E] unused
   int32_t* meta;      // [16] device scalars: [0] touched experts, [1] valid pairs, [2] token groups,
-                      //       [3] token chunks, [8] / [9] unit counters of the gate/up and down GEMMs
+                      //       [3] token chunks, [8] / [9] unit counters of the gate/up and down GEMMs,
+                      //       [10] finished CTAs of the fused decode top-k
   int32_t* group_base;  // [E + 1] first token group of each touched expert (touched order)
   int32_t* tile_base;   // [E + 1] first token chunk of each touched expert
   int32_t* sorted_pair;  // [P] pair id (t * k + slot) at each sorted position
@@ -119,8 +120,10 @@ cudaError_t launch_gemm_down(const moe_desc& d, const float* topk_w, const Works
 bool decode_route_ok(const moe_desc& d, int T);
 bool fused_route_sort_ok(const moe_desc& d, int T);
 int decode_logit_splits(const moe_desc& d, int T);  // S: partial sums per logit (1, 2, 4 or 8)
+// topk_done (optional): the fused top-k's completion counter, zeroed by this launch
+constexpr int kMetaTopkDone = 10;
 cudaError_t launch_decode_logits(const moe_desc& d, const void* x, int T, float* partial, int S, uint32_t* flags,
-                                 cudaStream_t s);
+                                 cudaStream_t s, int32_t* topk_done = nullptr);
 cudaError_t launch_topk_sort(const moe_desc& d, const float* partial, int S, int T, int32_t* idx, float* w,
                              int chunk, const Workspace& ws, uint32_t* flags, cudaStream_t s);
 cudaError_t launch_expert_counts(const int32_t* idx, int64_t n, int E, uint64_t* counts, int num_sms,

@@ -386,7 +386,8 @@ extern "C" moe_status moe_layer_forward(const moe_desc* d, const void* x, int32_
   if ((st = device_state(&dev)) != MOE_OK) return st;
   const Workspace ws = carve_workspace(*d, T, workspace);
   const int S = decode_logit_splits(*d, T);
-  MOE_LAUNCH("router_decode_logits", stream, launch_decode_logits(*d, x, T, ws.logits, S, dev->flags, stream));
+  MOE_LAUNCH("router_decode_logits", stream,
+             launch_decode_logits(*d, x, T, ws.logits, S, dev->flags, stream, ws.meta + kMetaTopkDone));
   MOE_LAUNCH("router_topk_sort", stream,
              launch_topk_sort(*d, ws.logits, S, T, topk_idx, topk_w, chunk_tokens(T, d->k, d->E), ws, dev->flags,
                               stream));

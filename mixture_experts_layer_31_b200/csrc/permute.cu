@@ -123,9 +123,9 @@ __global__ void __launch_bounds__(1024) small_sort_kernel(const int32_t* __restr
                                                           int32_t* __restrict__ meta,
                                                           int32_t* __restrict__ sorted_pair, uint32_t* flags) {
   __shared__ int32_t base[kSortWarps][kSmallE];
-  __shared__ int warp_sums[32];
+  __shared__ int4 warp_sums4[32];
   route_dev::block_small_sort(idx, P, E, chunk, counts, offsets, touched, group_base, tile_base, meta, sorted_pair,
-                              flags, base, warp_sums);
+                              flags, base, warp_sums4);
 }
 
 }  // namespace

@@ -146,86 +146,166 @@ __device__ __forceinline__ void warp_topk(const float* __restrict__ partial, int
   }
 }
 
-// Small batches: the whole sort in one CTA of 32 warps.  Warp w owns the
-// contiguous pair segment [w*seg, (w+1)*seg): it counts its pairs per expert
-// (no atomics: match_any groups equal experts, the last peer adds), the block
-// turns (warp, expert) counts into exclusive bases, and each warp re-walks its
+// Exclusive prefix sums of four values at once over the block (blockDim.x <=
+// 1024); the block totals go to *total.
+__device__ __forceinline__ int4 block_exclusive_scan4(int4 v, int4* warp_sums4, int4* total) {
+  const int lane = lane_id(), w = warp_id(), nw = blockDim.x >> 5;
+  int4 incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int nx = __shfl_up_sync(0xFFFFFFFFu, incl.x, off);
+    const int ny = __shfl_up_sync(0xFFFFFFFFu, incl.y, off);
+    const int nz = __shfl_up_sync(0xFFFFFFFFu, incl.z, off);
+    const int nw4 = __shfl_up_sync(0xFFFFFFFFu, incl.w, off);
+    if (lane >= off) {
+      incl.x += nx;
+      incl.y += ny;
+      incl.z += nz;
+      incl.w += nw4;
+    }
+  }
+  if (lane == 31) warp_sums4[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int4 s = lane < nw ? warp_sums4[lane] : make_int4(0, 0, 0, 0);
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int nx = __shfl_up_sync(0xFFFFFFFFu, s.x, off);
+      const int ny = __shfl_up_sync(0xFFFFFFFFu, s.y, off);
+      const int nz = __shfl_up_sync(0xFFFFFFFFu, s.z, off);
+      const int nw4 = __shfl_up_sync(0xFFFFFFFFu, s.w, off);
+      if (lane >= off) {
+        s.x += nx;
+        s.y += ny;
+        s.z += nz;
+        s.w += nw4;
+      }
+    }
+    if (lane < nw) warp_sums4[lane] = s;  // inclusive over warps
+  }
+  __syncthreads();
+  const int4 prev = w > 0 ? warp_sums4[w - 1] : make_int4(0, 0, 0, 0);
+  *total = warp_sums4[nw - 1];
+  __syncthreads();
+  return make_int4(prev.x + incl.x - v.x, prev.y + incl.y - v.y, prev.z + incl.z - v.z, prev.w + incl.w - v.w);
+}
+
+// Small batches: the whole sort in one CTA of 32 warps.  The P pairs are cut
+// into nseg <= 32 contiguous segments of whole 32-pair rounds; warp w < nseg
+// owns segment w: it loads its pairs' experts into registers (all loads in
+// flight at once), counts them per expert (no atomics: a ballot match groups equal
+// experts, the last peer adds), the block turns (segment, expert) counts into
+// exclusive bases with one four-way prefix scan, and each warp re-walks its
 // segment in order to scatter.  Same stable order as the chunked kernels.
 constexpr int kSmallE = 256;
 constexpr int kSortWarps = 32;
 
+// The lanes of the warp holding the same value as this lane, for values in
+// [-1, kSmallE): nine ballots over the bits of value + 1 (what __match_any_sync
+// returns, in a fixed handful of cheap instructions).
+__device__ __forceinline__ unsigned match_small(int v) {
+  static_assert(kSmallE <= 511, "nine bits");
+  const unsigned key = (unsigned)(v + 1);
+  unsigned peers = 0xFFFFFFFFu;
+#pragma unroll
+  for (int b = 0; b < 9; ++b) {
+    const bool bit = (key >> b) & 1u;
+    const unsigned m = __ballot_sync(0xFFFFFFFFu, bit);
+    peers &= bit ? m : ~m;
+  }
+  return peers;
+}
+constexpr int kSortRounds = 8;  // 32-pair rounds per segment: P <= kSortWarps * 32 * kSortRounds = 8192
+
 // Called by all threads of a CTA of kSortWarps warps; base and warp_sums are
-// shared memory of the caller ([kSortWarps][kSmallE] and [32] ints).
+// shared memory of the caller ([kSortWarps][kSmallE] ints and 4 x 32 ints,
+// 16-byte aligned).  P <= 8192, E <= kSmallE.
 __device__ __forceinline__ void block_small_sort(const int32_t* idx, int P, int E, int chunk,
                                                  int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                                                  int32_t* __restrict__ touched, int32_t* __restrict__ group_base,
                                                  int32_t* __restrict__ tile_base, int32_t* __restrict__ meta,
                                                  int32_t* __restrict__ sorted_pair, uint32_t* flags,
-                                                 int32_t (*base)[kSmallE], int* warp_sums) {
+                                                 int32_t (*base)[kSmallE], int4* warp_sums4) {
   const int w = warp_id(), lane = lane_id();
-  for (int i = threadIdx.x; i < kSortWarps * kSmallE; i += blockDim.x) (&base[0][0])[i] = 0;
-  __syncthreads();
-  const int seg = (P + kSortWarps - 1) / kSortWarps;
+  const int rounds = (P + 32 * kSortWarps - 1) / (32 * kSortWarps);  // per segment, <= kSortRounds
+  const int seg = 32 * (rounds > 0 ? rounds : 1);
+  const int nseg = (P + seg - 1) / seg;
+  for (int i = threadIdx.x; i < nseg * kSmallE; i += blockDim.x) (&base[0][0])[i] = 0;
   const int p0 = min(P, w * seg), p1 = min(P, p0 + seg);
-  const unsigned lt = (1u << lane) - 1u;
+  int ev[kSortRounds];
   bool bad = false;
-  for (int pb = p0; pb < p1; pb += 32) {
-    const int p = pb + lane;
-    int e = (p < p1) ? idx[p] : -1;
-    if (p < p1 && (e < 0 || e >= E)) bad = true;
+#pragma unroll
+  for (int r = 0; r < kSortRounds; ++r) {
+    const int p = p0 + 32 * r + lane;
+    int e = (r < rounds && p < p1) ? idx[p] : -1;
+    if (r < rounds && p < p1 && (e < 0 || e >= E)) bad = true;
     if (e < 0 || e >= E) e = -1;
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
-    if (e >= 0 && lane == 31 - __clz(peers)) base[w][e] += __popc(peers);
+    ev[r] = e;
+  }
+  __syncthreads();
+  const unsigned lt = (1u << lane) - 1u;
+  if (w < nseg) {
+#pragma unroll
+    for (int r = 0; r < kSortRounds; ++r) {
+      if (r < rounds) {
+        const int e = ev[r];
+        const unsigned peers = match_small(e);
+        if (e >= 0 && lane == 31 - __clz(peers)) base[w][e] += __popc(peers);
+        __syncwarp();
+      }
+    }
   }
   if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) raise_flag(flags, MOE_FLAG_BAD_EXPERT_INDEX);
   __syncthreads();
-  // per expert: exclusive prefix over warps, then over experts
+  // per expert: exclusive prefix over segments, then over experts
   const int e = threadIdx.x;
   int running = 0;
   if (e < E) {
-    for (int ww = 0; ww < kSortWarps; ++ww) {
+    for (int ww = 0; ww < nseg; ++ww) {
       const int v = base[ww][e];
       base[ww][e] = running;
       running += v;
     }
     counts[e] = running;
   }
-  int total;
-  const int off = block_exclusive_scan(e < E ? running : 0, warp_sums, &total);
+  const bool live = e < E && running > 0;
+  const int4 mine = make_int4(e < E ? running : 0, live ? 1 : 0,
+                              e < E ? (running + kGemvGroup - 1) / kGemvGroup : 0,
+                              e < E ? (running + chunk - 1) / chunk : 0);
+  int4 tot;
+  const int4 pos = block_exclusive_scan4(mine, warp_sums4, &tot);
+  // pos.x: offset, pos.y: position among touched experts, pos.z: first group, pos.w: first chunk
   if (e < E) {
-    offsets[e] = off;
-    for (int ww = 0; ww < kSortWarps; ++ww) base[ww][e] += off;
+    offsets[e] = pos.x;
+    for (int ww = 0; ww < nseg; ++ww) base[ww][e] += pos.x;
   }
-  if (e == 0) offsets[E] = total;
-  int ntouched;
-  const int tpos = block_exclusive_scan((e < E && running > 0) ? 1 : 0, warp_sums, &ntouched);
-  if (e < E && running > 0) touched[tpos] = e;
-  const int groups = (e < E) ? (running + kGemvGroup - 1) / kGemvGroup : 0;
-  int ngroups;
-  const int gpos = block_exclusive_scan(groups, warp_sums, &ngroups);
-  if (e < E && running > 0) group_base[tpos] = gpos;
-  const int chunks = (e < E) ? (running + chunk - 1) / chunk : 0;
-  int nchunks;
-  const int cpos = block_exclusive_scan(chunks, warp_sums, &nchunks);
-  if (e < E && running > 0) tile_base[tpos] = cpos;
+  if (live) {
+    touched[pos.y] = e;
+    group_base[pos.y] = pos.z;
+    tile_base[pos.y] = pos.w;
+  }
   if (e == 0) {
-    meta[0] = ntouched;
-    meta[1] = total;
-    meta[2] = ngroups;
-    meta[3] = nchunks;
-    group_base[ntouched] = ngroups;
-    tile_base[ntouched] = nchunks;
+    offsets[E] = tot.x;
+    meta[0] = tot.y;
+    meta[1] = tot.x;
+    meta[2] = tot.z;
+    meta[3] = tot.w;
+    group_base[tot.y] = tot.z;
+    tile_base[tot.y] = tot.w;
   }
   __syncthreads();
-  for (int pb = p0; pb < p1; pb += 32) {
-    const int p = pb + lane;
-    int ee = (p < p1) ? idx[p] : -1;
-    if (ee < 0 || ee >= E) ee = -1;
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, ee);
-    if (ee >= 0) sorted_pair[base[w][ee] + __popc(peers & lt)] = p;
-    __syncwarp();
-    if (ee >= 0 && lane == 31 - __clz(peers)) base[w][ee] += __popc(peers);
-    __syncwarp();
+  if (w < nseg) {
+#pragma unroll
+    for (int r = 0; r < kSortRounds; ++r) {
+      if (r < rounds) {
+        const int ee = ev[r];
+        const unsigned peers = match_small(ee);
+        if (ee >= 0) sorted_pair[base[w][ee] + __popc(peers & lt)] = p0 + 32 * r + lane;
+        __syncwarp();
+        if (ee >= 0 && lane == 31 - __clz(peers)) base[w][ee] += __popc(peers);
+        __syncwarp();
+      }
+    }
   }
 }
 

@@ -18,10 +18,10 @@
 //                         order.  Every sum's order depends on H (and T) only,
 //                         so a masked layer and its sliced twin get the same
 //                         logits bit for bit.  T <= 32.
-//   topk_sort_kernel      one CTA: top-k of every token (one warp per token),
-//                         then the stable counting sort by expert of all T*k
-//                         pairs -- the same device code as the standalone
-//                         kernels, without the launch in between.
+//   topk_sort_kernel      one CTA per token: its top-k (one warp); the CTA that
+//                         finishes last then runs the stable counting sort by
+//                         expert of all T*k pairs -- the same device code as the
+//                         standalone kernels, without the launch in between.
 #include "common.cuh"
 #include "internal.h"
 #include "route_dev.cuh"
@@ -49,8 +49,10 @@ template <bool XBF16>
 __global__ void __launch_bounds__(kLogitThreads) decode_logits_kernel(const void* __restrict__ x,
                                                                       const float* __restrict__ Wr, int T, int H,
                                                                       int E, int S, float* __restrict__ partial,
-                                                                      uint32_t* flags) {
+                                                                      int32_t* __restrict__ topk_done, uint32_t* flags) {
   extern __shared__ __align__(16) uint8_t smb[];
+  // the fused top-k launch that follows counts its finished CTAs from zero
+  if (topk_done != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *topk_done = 0;
   __shared__ __align__(8) uint64_t staged;
   const int len = H / S;                        // a multiple of 8
   const int sl = blockIdx.x % S, g = blockIdx.x / S;
@@ -136,13 +138,20 @@ __global__ void __launch_bounds__(kLogitThreads) decode_logits_kernel(const void
   }
 }
 
-// One CTA of 1024 threads, three phases with one global round trip:
-//   A  every thread sums the S partial logits of some (token, expert) pairs in
-//      the split order (split 0 first, as the standalone top-k does) into
-//      shared memory, and the bias and mask are staged there;
-//   B  one warp per token selects its top-k from shared memory (the same device
-//      code as the standalone top-k, so the routing is bit for bit the same);
-//   C  the stable counting sort reads the routing from shared memory.
+// One CTA of 1024 threads per token:
+//   A  the CTA sums its token's S partial logits of every expert in the split
+//      order (split 0 first, as the standalone top-k does) into shared memory
+//      and forms the keys (the same expressions as the standalone top-k);
+//   B  every selectable expert's rank among the selectable keys (key
+//      descending, expert index ascending -- the order in which the standalone
+//      top-k's repeated argmax picks them) is counted by four threads over a
+//      quarter of the experts each; ranks below k are the slots.  Warp 0 then
+//      renormalises exactly as the standalone top-k does (same values, same
+//      lanes, same butterfly), so the routing is bit for bit the same;
+//   C  the CTA that finishes last (a completion counter, zeroed by the logits
+//      kernel before this launch) reads every token's routing back and runs the
+//      stable counting sort, then re-arms the counter.
+// No CTA waits for another: the last one to arrive does the sort.
 // The logits and the sort's per-warp bases share one buffer (never live together).
 constexpr int kFusedMaxT = 32, kFusedMaxE = 256, kFusedMaxK = 32;
 
@@ -155,38 +164,104 @@ __global__ void __launch_bounds__(1024) topk_sort_kernel(const float* __restrict
                                                          int32_t* __restrict__ offsets, int32_t* __restrict__ touched,
                                                          int32_t* __restrict__ group_base,
                                                          int32_t* __restrict__ tile_base, int32_t* __restrict__ meta,
-                                                         int32_t* __restrict__ sorted_pair, uint32_t* flags) {
+                                                         int32_t* __restrict__ sorted_pair, int32_t* done,
+                                                         uint32_t* flags) {
   static_assert(kFusedMaxT * kFusedMaxE == route_dev::kSortWarps * route_dev::kSmallE, "shared buffer sizes");
   __shared__ __align__(16) int32_t buf[route_dev::kSortWarps][route_dev::kSmallE];  // logits, then sort bases
-  __shared__ float bias_s[kFusedMaxE];
-  __shared__ uint8_t mask_s[kFusedMaxE];
   __shared__ int32_t idx_s[kFusedMaxT * kFusedMaxK];
-  __shared__ int warp_sums[32];
-  float* logits = reinterpret_cast<float*>(&buf[0][0]);  // [T][E]
-  // A: partial sums, all loads of a thread in flight together
-  for (int i = threadIdx.x; i < T * E; i += blockDim.x) {
-    const int t = i / E, e = i - t * E;
+  __shared__ int4 warp_sums4[32];
+  __shared__ int sel_e[kFusedMaxE];     // selectable flags, then nothing
+  __shared__ int slot_e[kFusedMaxK];    // expert of each slot
+  __shared__ float slot_r[kFusedMaxK];  // its router value (sigmoid or logit)
+  __shared__ int last;
+  float* logits = reinterpret_cast<float*>(&buf[0][0]);  // [E] of this CTA's token
+  float* keys = logits + kFusedMaxE;                      // [E], -inf where not selectable
+  int32_t* rank_part = &buf[2][0];                        // [4][E] partial ranks
+  const int t = blockIdx.x;
+  const int tid = threadIdx.x;
+  // A
+  bool bad = false;
+  if (tid < E) {
     float p[S];
 #pragma unroll
-    for (int s = 0; s < S; ++s) p[s] = partial[((size_t)s * T + t) * E + e];
+    for (int s = 0; s < S; ++s) p[s] = partial[((size_t)s * T + t) * E + tid];
     float sum = 0.f;
 #pragma unroll
     for (int s = 0; s < S; ++s) sum += p[s];
-    logits[i] = sum;
+    logits[tid] = sum;
+    const bool active = (mask == nullptr) || (mask[tid] != 0);
+    float key = -INFINITY;
+    if (!isfinite(sum)) {
+      bad = true;
+    } else if (active) {
+      key = (router == MOE_ROUTER_SIGMOID_BIAS) ? sigmoidf_acc(sum) + (bias ? bias[tid] : 0.f) : sum;
+    }
+    keys[tid] = key;
+    // selectable: active, finite logit, and a key that compares (a NaN bias makes
+    // a key the standalone top-k can never pick)
+    sel_e[tid] = active && !bad && key == key ? 1 : 0;
   }
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    if (bias) bias_s[e] = bias[e];
-    if (mask) mask_s[e] = mask[e];
+  const int nsel = __syncthreads_count(tid < E && sel_e[tid] != 0);
+  if (__syncthreads_or(bad) && tid == 0) raise_flag(flags, MOE_FLAG_NONFINITE_LOGIT);
+  // B: partial ranks, four threads per expert
+  {
+    const int e = tid & (kFusedMaxE - 1), q = tid / kFusedMaxE;  // q in 0..3
+    if (e < E) {
+      int r = 0;
+      if (sel_e[e]) {
+        const float ke = keys[e];
+        const int lo = q * (kFusedMaxE / 4), hi = min(E, lo + kFusedMaxE / 4);
+        for (int j = lo; j < hi; ++j) r += (sel_e[j] && route_dev::better(keys[j], j, ke, e)) ? 1 : 0;
+      }
+      rank_part[q * kFusedMaxE + e] = r;
+    }
   }
   __syncthreads();
-  // B
-  for (int t = warp_id(); t < T; t += blockDim.x >> 5)
-    route_dev::warp_topk<PER_LANE, 1>(logits, T, t, E, k, router, bias ? bias_s : nullptr, mask ? mask_s : nullptr,
-                                      scale, idx, wout, flags, idx_s);
+  int slot = -1;
+  if (tid < E && sel_e[tid]) {
+    const int r = rank_part[tid] + rank_part[kFusedMaxE + tid] + rank_part[2 * kFusedMaxE + tid] +
+                  rank_part[3 * kFusedMaxE + tid];
+    if (r < k) slot = r;
+  }
+  __syncthreads();  // every thread has read the selectable flags
+  if (slot >= 0) {
+    slot_e[slot] = tid;
+    slot_r[slot] = (router == MOE_ROUTER_SIGMOID_BIAS) ? sigmoidf_acc(logits[tid]) : logits[tid];
+  }
   __syncthreads();
-  // C
+  if (warp_id() == 0) {
+    const int lane = lane_id();
+    int my_e = -1;
+    float my_r = 0.f;
+    if (lane < k && lane < nsel) {
+      my_e = slot_e[lane];
+      my_r = slot_r[lane];
+    }
+    if (nsel < k && lane == 0) raise_flag(flags, MOE_FLAG_TOO_FEW_ACTIVE);
+    // renormalise over the chosen slots (softmax: exp relative to the best logit)
+    const float top = __shfl_sync(0xFFFFFFFFu, my_r, 0);
+    float v = 0.f;
+    if (lane < k && my_e >= 0) v = (router == MOE_ROUTER_SIGMOID_BIAS) ? my_r : expf(my_r - top);
+    float total = v;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) total += __shfl_xor_sync(0xFFFFFFFFu, total, off);
+    if (lane < k) {
+      idx[(size_t)t * k + lane] = my_e;
+      wout[(size_t)t * k + lane] = (my_e >= 0 && total > 0.f) ? v / total * scale : 0.f;
+    }
+    __threadfence();  // this token's routing is visible device-wide before the count below
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(done, 1) == (int)gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  // C (the last CTA): every other CTA's routing is visible once its count is
+  __threadfence();
+  for (int i = threadIdx.x; i < T * k; i += blockDim.x) idx_s[i] = __ldcg(idx + i);
+  __syncthreads();
   route_dev::block_small_sort(idx_s, T * k, E, chunk, counts, offsets, touched, group_base, tile_base, meta,
-                              sorted_pair, flags, buf, warp_sums);
+                              sorted_pair, flags, buf, warp_sums4);
+  if (threadIdx.x == 0) *done = 0;
 }
 
 }  // namespace
@@ -216,22 +291,22 @@ int decode_logit_splits(const moe_desc& d, int T) {
 }
 
 cudaError_t launch_decode_logits(const moe_desc& d, const void* x, int T, float* partial, int S, uint32_t* flags,
-                                 cudaStream_t s) {
+                                 cudaStream_t s, int32_t* topk_done) {
   const dim3 grid(S * ((d.E + kGroupE - 1) / kGroupE));
   const bool xb = d.xfmt == MOE_X_BF16;
   const size_t smem = decode_logits_smem(d.H, T, S, xb);
   auto kern = xb ? decode_logits_kernel<true> : decode_logits_kernel<false>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  return launch_k(kern, grid, dim3(kLogitThreads), smem, s, x, d.W_r, T, d.H, d.E, S, partial, flags);
+  return launch_k(kern, grid, dim3(kLogitThreads), smem, s, x, d.W_r, T, d.H, d.E, S, partial, topk_done, flags);
 }
 
 cudaError_t launch_topk_sort(const moe_desc& d, const float* partial, int S, int T, int32_t* idx, float* w,
                              int chunk, const Workspace& ws, uint32_t* flags, cudaStream_t s) {
 #define MOE_TOPK_SORT(SS)                                                                                      \
-  return launch_k(topk_sort_kernel<8, SS>, dim3(1), dim3(1024), 0, s, partial, T, d.E, d.k, d.router, d.b,     \
+  return launch_k(topk_sort_kernel<8, SS>, dim3(T), dim3(1024), 0, s, partial, T, d.E, d.k, d.router, d.b,     \
                   d.expert_mask, d.scale, idx, w, chunk, ws.counts, ws.offsets, ws.touched, ws.group_base,    \
-                  ws.tile_base, ws.meta, ws.sorted_pair, flags)
+                  ws.tile_base, ws.meta, ws.sorted_pair, ws.meta + kMetaTopkDone, flags)
   switch (S) {
     case 1: MOE_TOPK_SORT(1);
     case 2: MOE_TOPK_SORT(2);
