@@ -299,6 +299,15 @@ typedef struct {
 MOE_API moe_status moe_stage_timing(int32_t enable);
 MOE_API moe_status moe_stage_times(moe_stage_time* out, int32_t capacity, int32_t* count);
 
+/*
+ * Restricts the per-kernel timing above to launches whose kernel name equals
+ * `name` (at most 31 characters; NULL or "" times every launch again).  Each
+ * timed launch adds two event records to its stream, and they cost time
+ * between kernels; timing one kernel keeps that cost off the others.
+ * Errors: MOE_ERR_INVALID_ARG if the name is too long.
+ */
+MOE_API moe_status moe_stage_timing_only(const char* name);
+
 #ifdef __cplusplus
 }
 #endif

@@ -40,7 +40,7 @@ EXPORTS = ("moe_workspace_size", "moe_route", "moe_forward", "moe_layer_forward"
            "moe_block_workspace_size",
            "moe_forward_block", "moe_expert_counts",
            "moe_cover_set", "moe_selftest_bounded_wait", "moe_last_error", "moe_device_flags", "moe_launch_count",
-           "moe_stage_timing", "moe_stage_times")
+           "moe_stage_timing", "moe_stage_times", "moe_stage_timing_only")
 MOE_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -97,10 +97,11 @@ def _load() -> ctypes.CDLL:
     lib.moe_launch_count.restype = ctypes.c_uint64
     lib.moe_stage_timing.argtypes = [i32]
     lib.moe_stage_times.argtypes = [ctypes.POINTER(moe_stage_time), i32, ctypes.POINTER(i32)]
+    lib.moe_stage_timing_only.argtypes = [ctypes.c_char_p]
     for f in ("moe_workspace_size", "moe_route", "moe_forward", "moe_layer_forward", "moe_forward_noalloc",
               "moe_block_workspace_size",
               "moe_forward_block", "moe_expert_counts",
-              "moe_cover_set", "moe_device_flags", "moe_stage_timing", "moe_stage_times"):
+              "moe_cover_set", "moe_device_flags", "moe_stage_timing", "moe_stage_times", "moe_stage_timing_only"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -208,6 +209,11 @@ def moe_launch_count() -> int:
 
 def moe_stage_timing(enable: bool) -> None:
     _check(lib().moe_stage_timing(1 if enable else 0))
+
+
+def moe_stage_timing_only(name=None) -> None:
+    """Time only the launches of kernel `name` (None: every launch again)."""
+    _check(lib().moe_stage_timing_only(None if not name else name.encode()))
 
 
 def moe_stage_times() -> dict:

@@ -76,6 +76,7 @@ static moe_status device_state(DeviceState** out) {
 
 static std::atomic<uint64_t> g_launches{0};
 static std::atomic<int> g_timing{0};
+static char g_timing_only[32] = {0};  // "" = every launch; guarded by g_time_mu
 
 struct Pending {
   char name[32];
@@ -102,6 +103,7 @@ void* launch_start(const char* name, cudaStream_t s) {
   nvtxRangePushA(name);
   if (!g_timing.load(std::memory_order_relaxed)) return nullptr;
   std::lock_guard<std::mutex> lk(g_time_mu);
+  if (g_timing_only[0] != 0 && strncmp(name, g_timing_only, sizeof(g_timing_only)) != 0) return nullptr;
   cudaEvent_t ev = pool_event();
   if (ev) cudaEventRecord(ev, s);
   return ev;
@@ -612,6 +614,15 @@ extern "C" uint64_t moe_launch_count(void) { return g_launches.load(); }
 
 extern "C" moe_status moe_stage_timing(int32_t enable) {
   g_timing.store(enable ? 1 : 0);
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_stage_timing_only(const char* name) {
+  g_err.clear();
+  if (name != nullptr && strlen(name) >= sizeof(g_timing_only))
+    return fail(MOE_ERR_INVALID_ARG, "kernel name longer than %d characters", (int)sizeof(g_timing_only) - 1);
+  std::lock_guard<std::mutex> lk(g_time_mu);
+  snprintf(g_timing_only, sizeof(g_timing_only), "%s", name ? name : "");
   return MOE_OK;
 }
 

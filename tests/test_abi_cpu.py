@@ -152,3 +152,13 @@ def test_block_workspace_covers_the_shared_expert():
     with pytest.raises(moe.MoeError) as ei:
         moe.moe_block_workspace_size(d, sh, 64)
     assert "shared expert" in str(ei.value)
+
+
+def test_stage_timing_filter_validates_the_name():
+    """Restricting the per-kernel timing to one kernel name needs no device;
+    names longer than the stage-name field are rejected."""
+    moe.moe_stage_timing_only("gemm_gateup")
+    moe.moe_stage_timing_only(None)
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_stage_timing_only("x" * 40)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG

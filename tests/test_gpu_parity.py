@@ -214,3 +214,14 @@ def test_stage_timing_reports_every_kernel(cid, T):
     sort = ("small_sort",) if "small_sort" in times else ("pair_histogram", "expert_scan", "pair_scatter")
     for name in sort:
         assert name in times and times[name][0] == 1 and times[name][1] > 0
+    # restricted to one kernel: only its launches are timed
+    moe.moe_stage_timing_only("combine")
+    moe.moe_stage_timing(True)
+    try:
+        layer(x)
+        layer(x)
+        only = moe.moe_stage_times()
+    finally:
+        moe.moe_stage_timing(False)
+        moe.moe_stage_timing_only(None)
+    assert set(only) == {"combine"} and only["combine"][0] == 2 and only["combine"][1] > 0
