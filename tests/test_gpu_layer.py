@@ -129,3 +129,40 @@ def test_zero_tokens_is_a_no_op_on_every_entry_point():
     torch.cuda.synchronize()
     assert moe.moe_launch_count() == n0
     assert int(counts.sum()) == 0
+
+
+@pytest.mark.parametrize("cid,over", [(2, {}), (3, dict(T=600, H=256, E=32, I=256))])
+def test_layer_replays_from_a_cuda_graph(cid, over):
+    """One moe_layer_forward call captured into a CUDA graph (no allocation, no
+    host synchronisation inside the call) replays to the same bits as a direct
+    call, and stays correct for new inputs written into the captured buffer."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    prob = synth.make_problem(cid, **over)
+    layer = layer_from_problem(prob)
+    x = x_to_device(prob)
+    y_ref, i_ref, w_ref = layer.layer(x)  # warm-up: device state, workspace, tensor maps
+    torch.cuda.synchronize()
+    xs = x.clone()
+    y = torch.empty_like(y_ref)
+    idx = torch.empty_like(i_ref)
+    w = torch.empty_like(w_ref)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer.layer(xs, out=(y, idx, w))
+    y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(idx, i_ref) and torch.equal(w, w_ref)
+    assert torch.equal(y.view(torch.int16) if y.dtype == torch.bfloat16 else y,
+                       y_ref.view(torch.int16) if y_ref.dtype == torch.bfloat16 else y_ref)
+    # new tokens in the captured input buffer: the replay routes and computes them
+    x2 = torch.roll(x, shifts=1, dims=0)
+    xs.copy_(x2)
+    g.replay()
+    y2, i2, w2 = layer.layer(x2)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, i2) and torch.equal(w, w2)
+    assert torch.equal(y.view(torch.int16) if y.dtype == torch.bfloat16 else y,
+                       y2.view(torch.int16) if y2.dtype == torch.bfloat16 else y2)
+    assert moe.moe_device_flags(clear=True) == 0
