@@ -85,6 +85,7 @@ struct GemmArgs {
   int S;
   int Hx;               // columns of x (the K coordinate of x is taken modulo Hx)
   int act;              // gate/up: moe_act (SiLU or tanh-GELU)
+  int out_bf16;         // down: the routed problem's per-pair outputs in bf16 (else fp32)
   int qsh;              // int4: log2 of the scale block (5: 32 columns, 7: 128)
   // optional second, dense problem in the same launch (the shared expert): every
   // one of Td tokens in token order with weight 1, expert 0 of weights with Rd rows
@@ -580,6 +581,12 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
           const int row = t.ib * Tr::kRows + tile * kBM + et;
           const float sd = WF == MOE_W_INT8_ROW ? pv.s0[(size_t)t.e * pv.R + row] : 1.f;
           float* yp = static_cast<float*>(pv.out);
+          uint16_t* yb = static_cast<uint16_t*>(pv.out);
+          const bool ob = a.out_bf16 && !t.dense;  // the dense problem's rows stay fp32
+          auto put = [&](int pair, float v) {
+            if (ob) yb[(size_t)pair * pv.R + row] = f32_to_bf16(v);
+            else yp[(size_t)pair * pv.R + row] = v;
+          };
           for (int n0 = c_first; n0 < t.n_tok; n0 += c_step) {
             uint32_t v[16];
             tmem_ld16(tacc + n0, v);
@@ -592,16 +599,15 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
               for (int j4 = 0; j4 < 4; ++j4) {
                 const int4 p = p4[j4];
                 const float4 wv = w4[j4];
-                yp[(size_t)p.x * pv.R + row] = wv.x * sd * __uint_as_float(v[4 * j4 + 0]);
-                yp[(size_t)p.y * pv.R + row] = wv.y * sd * __uint_as_float(v[4 * j4 + 1]);
-                yp[(size_t)p.z * pv.R + row] = wv.z * sd * __uint_as_float(v[4 * j4 + 2]);
-                yp[(size_t)p.w * pv.R + row] = wv.w * sd * __uint_as_float(v[4 * j4 + 3]);
+                put(p.x, wv.x * sd * __uint_as_float(v[4 * j4 + 0]));
+                put(p.y, wv.y * sd * __uint_as_float(v[4 * j4 + 1]));
+                put(p.z, wv.z * sd * __uint_as_float(v[4 * j4 + 2]));
+                put(p.w, wv.w * sd * __uint_as_float(v[4 * j4 + 3]));
               }
             } else {
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
-                if (n0 + j < t.n_tok)
-                  yp[(size_t)s_pair[n0 + j] * pv.R + row] = s_w[n0 + j] * sd * __uint_as_float(v[j]);
+                if (n0 + j < t.n_tok) put(s_pair[n0 + j], s_w[n0 + j] * sd * __uint_as_float(v[j]));
               }
             }
           }
@@ -974,7 +980,7 @@ cudaError_t launch_gemm_gateup(const moe_desc& d, const Workspace& ws, int P, in
 }
 
 cudaError_t launch_gemm_down(const moe_desc& d, const float* topk_w, const Workspace& ws, int P, int chunk,
-                             int num_sms, uint32_t* flags, cudaStream_t s, const DenseGemm* dg) {
+                             int num_sms, uint32_t* flags, cudaStream_t s, const DenseGemm* dg, bool yp_bf16) {
   Maps m;
   cudaError_t e = weight_map(&m.w0, d.W_down, d.wfmt, d.E, d.H, d.I, 128);
   if (e == cudaSuccess)
@@ -985,6 +991,7 @@ cudaError_t launch_gemm_down(const moe_desc& d, const float* topk_w, const Works
   a.s0 = d.s_down;
   a.topk_w = topk_w;
   a.out = ws.yp;
+  a.out_bf16 = yp_bf16 ? 1 : 0;
   a.R = d.H;
   a.K = d.I;
   a.qsh = d.wfmt == MOE_W_INT4_B128 ? 7 : 5;

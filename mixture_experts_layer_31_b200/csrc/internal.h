@@ -58,6 +58,7 @@ struct Workspace {
   int32_t* sorted_pair;  // [P] pair id (t * k + slot) at each sorted position
   void* hbuf;         // [P, I] activations between the two projections (bf16, or fp32 for fp32 weights)
   float* yp;          // [P, H] per-pair expert outputs times routing weight, indexed by pair id
+                      //         (fp32; bf16 -- in the first half of the area -- when yp_bf16())
   void* xs;           // [P, H] bf16 tokens gathered in sorted order (tensor-core path)
   void* w3;           // [E, 3H] bf16 three-way split of W_r (tensor-core router)
   size_t total;
@@ -114,7 +115,16 @@ struct DenseGemm {
 cudaError_t launch_gemm_gateup(const moe_desc& d, const Workspace& ws, int P, int chunk, int num_sms,
                                uint32_t* flags, cudaStream_t s, const DenseGemm* dg = nullptr);
 cudaError_t launch_gemm_down(const moe_desc& d, const float* topk_w, const Workspace& ws, int P, int chunk,
-                             int num_sms, uint32_t* flags, cudaStream_t s, const DenseGemm* dg = nullptr);
+                             int num_sms, uint32_t* flags, cudaStream_t s, const DenseGemm* dg = nullptr,
+                             bool yp_bf16 = false);
+// Large bf16 batches on the tensor-core path keep the per-pair expert outputs in
+// bf16 (fp32 accumulation, one rounding): half the down projection's output
+// bytes and half the combine's reads, where that traffic is a visible share of
+// the layer.  Smaller batches keep them in fp32.
+constexpr int kYpBf16MinT = 2048;
+inline bool yp_bf16(const moe_desc& d, int T, int path) {
+  return path == MOE_PATH_GEMM && d.xfmt == MOE_X_BF16 && T >= kYpBf16MinT;
+}
 // decode-sized batches (T <= 32): fp32 logits in one launch; with E <= 256 and
 // T*k <= 8192 also top-k and the expert sort in one launch
 bool decode_route_ok(const moe_desc& d, int T);
@@ -128,7 +138,7 @@ cudaError_t launch_topk_sort(const moe_desc& d, const float* partial, int S, int
                              int chunk, const Workspace& ws, uint32_t* flags, cudaStream_t s);
 cudaError_t launch_expert_counts(const int32_t* idx, int64_t n, int E, uint64_t* counts, int num_sms,
                                  cudaStream_t s);
-cudaError_t launch_combine(const moe_desc& d, const int32_t* idx, int T, const float* yp, void* y,
+cudaError_t launch_combine(const moe_desc& d, const int32_t* idx, int T, const void* yp, bool yp_bf16, void* y,
                            cudaStream_t s, const float* ys = nullptr, const void* residual = nullptr);
 cudaError_t launch_dense_plan(int T, int chunk, int32_t* counts, int32_t* offsets, int32_t* touched,
                               int32_t* group_base, int32_t* tile_base, int32_t* meta, int32_t* sorted_pair,

@@ -301,7 +301,7 @@ extern "C" moe_status moe_route(const moe_desc* d, const void* x, int32_t T, int
 }
 
 // the routed experts: expert-sorted order (unless already built), gate/up, down;
-// leaves w * FFN rows in ws.yp
+// leaves w * FFN rows in ws.yp (bf16 when yp_bf16(*d, T, path), else fp32)
 static moe_status run_routed(const moe_desc* d, const void* x, int32_t T, const int32_t* topk_idx,
                              const float* topk_w, const Workspace& ws, int path, DeviceState* dev,
                              cudaStream_t stream, bool sorted = false, const DenseGemm* dense_up = nullptr,
@@ -327,7 +327,8 @@ static moe_status run_routed(const moe_desc* d, const void* x, int32_t T, const 
     MOE_LAUNCH("gemm_gateup", stream,
                launch_gemm_gateup(*d, ws, P, chunk, dev->num_sms, dev->flags, stream, dense_up));
     MOE_LAUNCH("gemm_down", stream,
-               launch_gemm_down(*d, topk_w, ws, P, chunk, dev->num_sms, dev->flags, stream, dense_down));
+               launch_gemm_down(*d, topk_w, ws, P, chunk, dev->num_sms, dev->flags, stream, dense_down,
+                                yp_bf16(*d, T, path)));
   } else {
     MOE_LAUNCH("gemv_gateup", stream, launch_gemv_gateup(*d, x, d->k, ws, dev->num_sms, dev->flags, stream));
     MOE_LAUNCH("gemv_down", stream, launch_gemv_down(*d, topk_w, d->k, ws, dev->num_sms, dev->flags, stream));
@@ -362,7 +363,7 @@ extern "C" moe_status moe_forward(const moe_desc* d, const void* x, int32_t T, c
   if ((st = device_state(&dev)) != MOE_OK) return st;
   const Workspace ws = carve_workspace(*d, T, workspace);
   if ((st = run_routed(d, x, T, topk_idx, topk_w, ws, path, dev, stream)) != MOE_OK) return st;
-  MOE_LAUNCH("combine", stream, launch_combine(*d, topk_idx, T, ws.yp, y, stream));
+  MOE_LAUNCH("combine", stream, launch_combine(*d, topk_idx, T, ws.yp, yp_bf16(*d, T, path), y, stream));
   return MOE_OK;
 }
 
@@ -394,7 +395,7 @@ extern "C" moe_status moe_layer_forward(const moe_desc* d, const void* x, int32_
              launch_topk_sort(*d, ws.logits, S, T, topk_idx, topk_w, chunk_tokens(T, d->k, d->E), ws, dev->flags,
                               stream));
   if ((st = run_routed(d, x, T, topk_idx, topk_w, ws, path, dev, stream, true)) != MOE_OK) return st;
-  MOE_LAUNCH("combine", stream, launch_combine(*d, topk_idx, T, ws.yp, y, stream));
+  MOE_LAUNCH("combine", stream, launch_combine(*d, topk_idx, T, ws.yp, yp_bf16(*d, T, path), y, stream));
   return MOE_OK;
 }
 
@@ -493,7 +494,8 @@ extern "C" moe_status moe_forward_block(const moe_desc* d, const moe_shared_expe
     const DenseGemm up{&sd, x, ss.hbuf, T, chunk};
     const DenseGemm down{&sd, ss.hbuf, ss.yp, T, chunk};
     if ((st = run_routed(d, x, T, topk_idx, topk_w, ws, path, dev, stream, false, &up, &down)) != MOE_OK) return st;
-    MOE_LAUNCH("combine", stream, launch_combine(*d, topk_idx, T, ws.yp, y, stream, ss.yp, residual));
+    MOE_LAUNCH("combine", stream,
+               launch_combine(*d, topk_idx, T, ws.yp, yp_bf16(*d, T, path), y, stream, ss.yp, residual));
     return MOE_OK;
   }
   if ((st = run_routed(d, x, T, topk_idx, topk_w, ws, path, dev, stream)) != MOE_OK) return st;
@@ -514,7 +516,8 @@ extern "C" moe_status moe_forward_block(const moe_desc* d, const moe_shared_expe
     }
     ys = ss.yp;
   }
-  MOE_LAUNCH("combine", stream, launch_combine(*d, topk_idx, T, ws.yp, y, stream, ys, residual));
+  MOE_LAUNCH("combine", stream,
+             launch_combine(*d, topk_idx, T, ws.yp, yp_bf16(*d, T, path), y, stream, ys, residual));
   return MOE_OK;
 }
 

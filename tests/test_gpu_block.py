@@ -24,6 +24,7 @@ CASES = {
     "shared-only": (3, dict(T=64, H=256, E=16, I=128, shared=128)),
     "residual-only": (2, dict(T=33, H=256, E=16, I=128, residual=True)),
     "large-T-chunks": (3, dict(T=1500, H=256, E=16, I=128, shared=256, residual=True)),
+    "bf16-yp": (3, dict(T=2100, H=256, E=16, I=128, shared=256, residual=True)),  # routed rows in bf16
 }
 
 
@@ -68,8 +69,9 @@ def test_block_prefill_sampled():
     judge_block(prob, y, idx, w, tokens=np.unique(np.concatenate([[0, prob.T - 1], rng.choice(prob.T, 30)])))
 
 
-def test_block_without_extras_equals_forward_bit_for_bit():
-    prob = synth.make_problem(3, T=300, H=256, E=16, I=128)
+@pytest.mark.parametrize("T", [300, 2100])
+def test_block_without_extras_equals_forward_bit_for_bit(T):
+    prob = synth.make_problem(3, T=T, H=256, E=16, I=128)
     layer = layer_from_problem(prob)
     x = x_to_device(prob)
     idx, w = layer.route(x)

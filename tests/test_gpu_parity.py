@@ -32,6 +32,9 @@ SMALL = {
     "tiny-fp32-gelu": (1, dict(act="gelu_tanh")),
     "qwen3-int4b128-small": (4, dict(T=150, H=256, E=16, I=256, wfmt="int4b128")),
     "qwen3-int4b128-gelu": (4, dict(T=77, H=384, E=12, I=128, wfmt="int4b128", act="gelu_tanh")),
+    # T >= 2048 on the tensor cores: per-pair outputs kept in bf16 before the combine
+    "kimi-int8-bf16-yp": (3, dict(T=2100, H=256, E=16, I=128)),
+    "qwen3-int4-bf16-yp": (4, dict(T=2048, H=256, E=16, I=256)),
 }
 
 
