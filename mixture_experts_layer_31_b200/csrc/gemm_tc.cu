@@ -837,12 +837,27 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
     meta[9] = 0;
   }
   const int P = meta[1];
-  const int per_row = H / 8;  // 16-byte chunks
-  const size_t n = (size_t)P * per_row;
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
-    const int pos = (int)(i / per_row), c = (int)(i - (size_t)pos * per_row) * 8;
+  // a warp copies a 128-chunk segment of one row (16-byte chunks): lane l takes
+  // chunks l, l+32, l+64, l+96, all four loads in flight before the stores, and
+  // every load and store instruction covers 512 contiguous bytes
+  const int lane = threadIdx.x & 31;
+  const int per_row = H / 8;
+  const int nseg = (per_row + 127) / 128;
+  const size_t items = (size_t)P * nseg;
+  const size_t nwarps = ((size_t)gridDim.x * blockDim.x) >> 5;
+  for (size_t it = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items; it += nwarps) {
+    const int pos = (int)(it / nseg), seg = (int)(it - (size_t)pos * nseg);
     const int t = sorted_pair[pos] / k;
-    *reinterpret_cast<uint4*>(xs + (size_t)pos * H + c) = *reinterpret_cast<const uint4*>(x + (size_t)t * H + c);
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+    uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)pos * H);
+    const int c0 = seg * 128 + lane;
+    uint4 v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (c0 + 32 * q < per_row) v[q] = src[c0 + 32 * q];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (c0 + 32 * q < per_row) dst[c0 + 32 * q] = v[q];
   }
 }
 
@@ -931,8 +946,8 @@ bool gemm_tc_supported(const moe_desc& d) {
 
 cudaError_t launch_gather_rows(const moe_desc& d, const void* x, const Workspace& ws, int P, int num_sms,
                                cudaStream_t s) {
-  const size_t n = (size_t)P * (d.H / 8);
-  int blocks = (int)((n + 255) / 256);
+  const size_t warps = (size_t)P * ((d.H / 8 + 127) / 128);  // one warp per 128-chunk row segment
+  int blocks = (int)((warps + 7) / 8);
   if (blocks > num_sms * 8) blocks = num_sms * 8;
   if (blocks < 1) blocks = 1;
   return launch_k(gather_rows_kernel, dim3(blocks), dim3(256), 0, s, static_cast<const uint16_t*>(x), d.H, d.k,
