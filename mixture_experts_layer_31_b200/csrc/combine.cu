@@ -17,6 +17,8 @@ template <bool OUT_BF16, bool EXTRA>
 __global__ void __launch_bounds__(256) combine_kernel(const int32_t* __restrict__ idx, int T, int H, int E,
                                                       int k, const float* __restrict__ yp,
                                                       const float* __restrict__ ys, const void* res, void* y) {
+  pdl_wait();
+  pdl_trigger();
   // res and y may alias (an in-place residual update): each element is read,
   // then written, by the same thread
   const int h4 = H / 4;
@@ -89,6 +91,8 @@ template <bool EXTRA>
 __global__ void __launch_bounds__(256) combine_bf16_kernel(const int32_t* __restrict__ idx, int T, int H, int E,
                                                            int k, const uint16_t* __restrict__ yp,
                                                            const float* __restrict__ ys, const void* res, void* y) {
+  pdl_wait();
+  pdl_trigger();
   const int h8 = H / 8;
   const size_t n = (size_t)T * h8;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {

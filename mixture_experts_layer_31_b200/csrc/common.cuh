@@ -66,6 +66,12 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
 }
 
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
+
+// Programmatic dependent launch (see launch_k): wait until the previous kernel
+// on the stream has finished and its writes are visible (a no-op when this
+// launch was not programmatic), and let the next kernel start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
 // ---------------------------------------------------------------- mbarrier + bulk copy (sm_90+/sm_100)

@@ -334,6 +334,10 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the prologue above touches only this CTA's shared memory, TMEM and the tensor
+  // maps; everything below reads what earlier launches wrote
+  pdl_wait();
+  pdl_trigger();
 
   const int ntouched = MODE == 2 ? 0 : a.meta[0];
   const int nib = (a.R + Tr::kRows - 1) / Tr::kRows;  // gate/up: the last block may be half (I % 128 == 64)
@@ -832,6 +836,8 @@ GemmArgs common(const Workspace& ws, int chunk, uint32_t* flags) {
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x, int H, int k,
                                                           const int32_t* __restrict__ sorted_pair,
                                                           int32_t* __restrict__ meta, uint16_t* __restrict__ xs) {
+  pdl_wait();
+  pdl_trigger();
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     meta[8] = 0;
     meta[9] = 0;
@@ -866,6 +872,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
 // relative, so bf16 x against W3 over 3H columns gives fp32-accurate logits
 __global__ void __launch_bounds__(256) split3_kernel(const float* __restrict__ Wr, int E, int H,
                                                      uint16_t* __restrict__ W3) {
+  pdl_wait();
+  pdl_trigger();
   const int q4 = H / 4;  // float4 quads per row
   const int n = E * q4;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {

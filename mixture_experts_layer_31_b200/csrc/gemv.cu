@@ -196,6 +196,8 @@ __device__ __forceinline__ void dot_piece(const uint32_t (&rows)[NW], const floa
 // MODE 0: gate/up (2 rows of each matrix per warp); MODE 1: down (4 rows per warp)
 template <int MODE, int WF, bool IN_BF16, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const StreamArgs a) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int NMAT = MODE == 0 ? 2 : 1;
   constexpr int RPW = MODE == 0 ? 2 : 4;

@@ -8,12 +8,29 @@
 
 namespace moe {
 
-// Launch one kernel on stream s (plain stream ordering) and report the launch status.
+// Programmatic dependent launch: every kernel of this library may start while
+// the kernel before it on the stream is finishing (its CTAs take SMs as they free
+// up and run their prologue); each waits (griddepcontrol.wait) before it reads
+// anything an earlier launch wrote, so results do not change.  MOE_PDL=0 in the
+// environment turns it off (plain stream ordering).
+bool pdl_enabled();
+
+// Launch one kernel on stream s and report the launch status.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                      Args&&... args) {
-  kernel<<<grid, block, smem, s>>>(static_cast<KArgs>(args)...);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // Tokens are routed in chunks of this many (token, slot) pairs when building

@@ -6,6 +6,7 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -76,6 +77,14 @@ static moe_status device_state(DeviceState** out) {
 
 static std::atomic<uint64_t> g_launches{0};
 static std::atomic<int> g_timing{0};
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("MOE_PDL");
+    return !(v != nullptr && v[0] == '0');
+  }();
+  return on;
+}
 static char g_timing_only[32] = {0};  // "" = every launch; guarded by g_time_mu
 
 struct Pending {
@@ -573,6 +582,8 @@ namespace {
 // one thread waits on an mbarrier that nothing completes: the library's bounded
 // wait gives up, the kernel raises MOE_FLAG_TIMEOUT and returns
 __global__ void bounded_wait_selftest_kernel(uint32_t* flags) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ __align__(8) uint64_t never;
   if (threadIdx.x == 0) {
     mbar_init(&never, 1);

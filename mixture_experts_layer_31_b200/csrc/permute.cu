@@ -18,6 +18,8 @@ namespace {
 __global__ void __launch_bounds__(256) pair_histogram_kernel(const int32_t* __restrict__ idx, int P, int E,
                                                              int32_t* __restrict__ chunk_hist,
                                                              uint32_t* flags) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int32_t hist[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
@@ -43,6 +45,8 @@ __global__ void __launch_bounds__(1024) expert_scan_kernel(int NC, int E, int32_
                                                            int32_t* __restrict__ group_base,
                                                            int32_t* __restrict__ tile_base, int chunk,
                                                            int32_t* __restrict__ meta) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int warp_sums[32];
   const int e = threadIdx.x;
   int running = 0;
@@ -88,6 +92,8 @@ __global__ void __launch_bounds__(1024) expert_scan_kernel(int NC, int E, int32_
 __global__ void __launch_bounds__(128) pair_scatter_kernel(const int32_t* __restrict__ idx, int P, int E,
                                                            const int32_t* __restrict__ chunk_base,
                                                            int32_t* __restrict__ sorted_pair) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int32_t running_all[];
   const int w = warp_id(), lane = lane_id();
   const int c = blockIdx.x * (blockDim.x >> 5) + w;
@@ -122,6 +128,8 @@ __global__ void __launch_bounds__(1024) small_sort_kernel(const int32_t* __restr
                                                           int32_t* __restrict__ tile_base,
                                                           int32_t* __restrict__ meta,
                                                           int32_t* __restrict__ sorted_pair, uint32_t* flags) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int32_t base[kSortWarps][kSmallE];
   __shared__ int4 warp_sums4[32];
   route_dev::block_small_sort(idx, P, E, chunk, counts, offsets, touched, group_base, tile_base, meta, sorted_pair,
@@ -161,6 +169,8 @@ __global__ void __launch_bounds__(256) dense_plan_kernel(int T, int chunk, int32
                                                          int32_t* __restrict__ group_base,
                                                          int32_t* __restrict__ tile_base, int32_t* __restrict__ meta,
                                                          int32_t* __restrict__ sorted_pair, float* __restrict__ ones) {
+  pdl_wait();
+  pdl_trigger();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < T; i += gridDim.x * blockDim.x) {
     sorted_pair[i] = i;
     ones[i] = 1.0f;

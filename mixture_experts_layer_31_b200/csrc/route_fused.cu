@@ -50,6 +50,8 @@ __global__ void __launch_bounds__(kLogitThreads) decode_logits_kernel(const void
                                                                       const float* __restrict__ Wr, int T, int H,
                                                                       int E, int S, float* __restrict__ partial,
                                                                       int32_t* __restrict__ topk_done, uint32_t* flags) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) uint8_t smb[];
   // the fused top-k launch that follows counts its finished CTAs from zero
   if (topk_done != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *topk_done = 0;
@@ -166,6 +168,8 @@ __global__ void __launch_bounds__(1024) topk_sort_kernel(const float* __restrict
                                                          int32_t* __restrict__ tile_base, int32_t* __restrict__ meta,
                                                          int32_t* __restrict__ sorted_pair, int32_t* done,
                                                          uint32_t* flags) {
+  pdl_wait();
+  pdl_trigger();
   static_assert(kFusedMaxT * kFusedMaxE == route_dev::kSortWarps * route_dev::kSmallE, "shared buffer sizes");
   __shared__ __align__(16) int32_t buf[route_dev::kSortWarps][route_dev::kSmallE];  // logits, then sort bases
   __shared__ int32_t idx_s[kFusedMaxT * kFusedMaxK];

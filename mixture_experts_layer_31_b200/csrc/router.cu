@@ -39,6 +39,8 @@ template <bool XBF16>
 __global__ void __launch_bounds__(256) router_logits_kernel(const void* __restrict__ x,
                                                             const float* __restrict__ Wr, int T, int H,
                                                             int E, int kc, float* __restrict__ partial) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ __align__(16) float xs[kBK][kBT + 4];
   __shared__ __align__(16) float wsm[kBK][kBE + 4];
   const int t0 = blockIdx.x * kBT, e0 = blockIdx.y * kBE, s = blockIdx.z;
@@ -127,6 +129,8 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
                                                           const uint8_t* __restrict__ mask, float scale,
                                                           int32_t* __restrict__ idx, float* __restrict__ wout,
                                                           uint32_t* flags) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x * (blockDim.x >> 5) + warp_id();
   if (t >= T) return;
   route_dev::warp_topk<PER_LANE, S>(partial, T, t, E, k, router, bias, mask, scale, idx, wout, flags);

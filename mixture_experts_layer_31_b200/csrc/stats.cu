@@ -14,6 +14,8 @@ constexpr int kCountThreads = 512;
 // block histogram in shared memory, then one 64-bit add per non-empty bin
 __global__ void __launch_bounds__(kCountThreads) expert_counts_kernel(const int32_t* __restrict__ idx, int64_t n,
                                                                       int E, unsigned long long* __restrict__ counts) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ uint32_t hist[1024];
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0u;
   __syncthreads();
