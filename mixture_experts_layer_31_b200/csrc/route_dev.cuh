@@ -1,7 +1,7 @@
 // Device-side pieces of the routing shared by the kernels that route, sort,
-// or do both in one launch: the warp-per-token top-k, the block prefix scan and
-// the single-CTA stable counting sort by expert.  Header-only so that every
-// kernel runs the same instructions.
+// or do both in one launch: the warp-per-token top-k, the block prefix scans and
+// the one-CTA stable counting sort by expert.  Header-only so that every kernel
+// runs the same instructions.
 #pragma once
 #include <math.h>
 
@@ -47,12 +47,11 @@ __device__ __forceinline__ bool better(float ka, int ea, float kb, int eb) {
 // Top-k of token t by one warp: sums the S partial logits of every expert in a
 // fixed order, forms the keys, selects k by repeated warp argmax (key
 // descending, expert index ascending) and writes the renormalised weights.
-// idx_copy (optional, e.g. shared memory) receives the selected experts too.
 template <int PER_LANE, int S>
 __device__ __forceinline__ void warp_topk(const float* __restrict__ partial, int T, int t, int E, int k, int router,
                                           const float* __restrict__ bias, const uint8_t* __restrict__ mask,
                                           float scale, int32_t* __restrict__ idx, float* __restrict__ wout,
-                                          uint32_t* flags, int32_t* idx_copy = nullptr) {
+                                          uint32_t* flags) {
   const int lane = lane_id();
   float logit[PER_LANE], key[PER_LANE];
   uint32_t avail = 0;
@@ -141,7 +140,6 @@ __device__ __forceinline__ void warp_topk(const float* __restrict__ partial, int
   for (int off = 16; off > 0; off >>= 1) total += __shfl_xor_sync(0xFFFFFFFFu, total, off);
   if (lane < k) {
     idx[(size_t)t * k + lane] = my_e;
-    if (idx_copy) idx_copy[t * k + lane] = my_e;
     wout[(size_t)t * k + lane] = (my_e >= 0 && total > 0.f) ? v / total * scale : 0.f;
   }
 }

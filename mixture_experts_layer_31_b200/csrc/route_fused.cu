@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(kLogitThreads) decode_logits_kernel(const void
 // The logits and the sort's per-warp bases share one buffer (never live together).
 constexpr int kFusedMaxT = 32, kFusedMaxE = 256, kFusedMaxK = 32;
 
-template <int PER_LANE, int S>
+template <int PER_LANE, int S>  // 32 * PER_LANE experts at most; S partial sums per logit
 __global__ void __launch_bounds__(1024) topk_sort_kernel(const float* __restrict__ partial, int T, int E, int k,
                                                          int router, const float* __restrict__ bias,
                                                          const uint8_t* __restrict__ mask, float scale,
@@ -171,6 +171,7 @@ __global__ void __launch_bounds__(1024) topk_sort_kernel(const float* __restrict
   pdl_wait();
   pdl_trigger();
   static_assert(kFusedMaxT * kFusedMaxE == route_dev::kSortWarps * route_dev::kSmallE, "shared buffer sizes");
+  static_assert(32 * PER_LANE >= kFusedMaxE, "experts per launch");
   __shared__ __align__(16) int32_t buf[route_dev::kSortWarps][route_dev::kSmallE];  // logits, then sort bases
   __shared__ int32_t idx_s[kFusedMaxT * kFusedMaxK];
   __shared__ int4 warp_sums4[32];
