@@ -92,6 +92,8 @@ def test_layer_forward_launches_fewer_kernels_at_decode():
 
 EDGE = {
     "max-H-decode": (2, dict(T=32, H=8192, E=16, I=64)),       # decode logits split 8 ways (213 KB of smem)
+    "max-E-decode": (2, dict(T=24, H=256, E=1024, I=64)),      # E > 256: route and forward, not the fused router
+    "max-k-decode": (2, dict(T=32, H=256, E=64, I=64, k=32)),  # 1024 pairs through the fused router's sort
     "max-I-decode": (2, dict(T=8, H=256, E=8, I=8192)),
     "k1-decode": (3, dict(T=17, H=256, E=24, I=128, k=1)),
     "k-equals-active": (5, dict(T=12, H=256, E=32, I=128, n_active=8, bias=("skew", 0.1))),

@@ -35,6 +35,10 @@ SMALL = {
     # T >= 2048 on the tensor cores: per-pair outputs kept in bf16 before the combine
     "kimi-int8-bf16-yp": (3, dict(T=2100, H=256, E=16, I=128)),
     "qwen3-int4-bf16-yp": (4, dict(T=2048, H=256, E=16, I=256)),
+    # the documented limits: E = 1024 experts, k = 32 slots
+    "kimi-int8-max-E": (3, dict(T=200, H=256, E=1024, I=128)),
+    "kimi-bf16-max-k": (2, dict(T=50, H=256, E=64, I=128, k=32)),
+    "qwen3-int4-max-E-max-k": (4, dict(T=90, H=256, E=1024, I=128, k=32)),
 }
 
 
@@ -57,7 +61,11 @@ def test_small_workloads(name, path):
         return
     _, _, y, idx, w = run(prob, PATHS[path])
     rep = judge(prob, y, idx, w)
-    assert rep["near_ties"] <= max(2, prob.T // 20)
+    # near-ties (k-th and (k+1)-th keys within 1e-4) are judged under the GPU's own
+    # routing after checking it is a valid top-k; they should be rare, except with
+    # 1024 experts, where the keys crowd together (a softmax over 1024 experts puts
+    # most probabilities within 1e-4 of each other)
+    assert rep["near_ties"] <= (prob.T if prob.E >= 512 else max(2, prob.T // 20))
 
 
 def test_tiny_fp32_full_tolerance():
