@@ -168,3 +168,39 @@ def test_layer_replays_from_a_cuda_graph(cid, over):
     assert torch.equal(y.view(torch.int16) if y.dtype == torch.bfloat16 else y,
                        y2.view(torch.int16) if y2.dtype == torch.bfloat16 else y2)
     assert moe.moe_device_flags(clear=True) == 0
+
+
+def test_programmatic_launch_does_not_change_results(tmp_path):
+    """The same layer calls with programmatic dependent launch (the default) and
+    with plain stream ordering (MOE_PDL=0, read once per process, so in a child
+    process) give the same bits."""
+    import os
+    import subprocess
+    import sys
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    here = os.path.dirname(os.path.abspath(__file__))
+    script = tmp_path / "run_layer.py"
+    script.write_text(
+        "import sys, numpy as np, torch\n"
+        f"sys.path[:0] = [{os.path.dirname(here)!r}, {here!r}]\n"
+        "import synth\n"
+        "from gpu_util import layer_from_problem, x_to_device\n"
+        "out = {}\n"
+        "for cid, over in ((2, {}), (3, dict(T=300, H=256, E=16, I=128)), (4, dict(T=150, H=256, E=16, I=128))):\n"
+        "    prob = synth.make_problem(cid, **over)\n"
+        "    layer = layer_from_problem(prob)\n"
+        "    y, idx, w = layer.layer(x_to_device(prob))\n"
+        "    torch.cuda.synchronize()\n"
+        "    out[f'y{cid}'] = y.view(torch.int16).cpu().numpy() if y.dtype == torch.bfloat16 else y.cpu().numpy()\n"
+        "    out[f'i{cid}'] = idx.cpu().numpy()\n"
+        "    out[f'w{cid}'] = w.cpu().numpy()\n"
+        "np.savez(sys.argv[1], **out)\n")
+    runs = {}
+    for pdl in ("1", "0"):
+        dst = tmp_path / f"out_{pdl}.npz"
+        env = dict(os.environ, MOE_PDL=pdl)
+        subprocess.run([sys.executable, str(script), str(dst)], check=True, env=env, timeout=600)
+        runs[pdl] = np.load(dst)
+    for key in runs["1"].files:
+        assert np.array_equal(runs["1"][key], runs["0"][key]), key
