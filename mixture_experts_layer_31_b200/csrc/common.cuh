@@ -25,6 +25,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// Two fp32 lanes at once (sm_100 paired fp32 arithmetic, round to nearest even
+// like the scalar instructions): (a + c) * s for a pair of fp32 bit patterns a,
+// with c and s applied to both lanes.
+__device__ __forceinline__ void add_mul_f32x2(uint32_t a0, uint32_t a1, float c, float s, float& r0, float& r1) {
+  asm("{\n\t.reg .b64 x, k, m;\n\t"
+      "mov.b64 x, {%2, %3};\n\t"
+      "mov.b64 k, {%4, %4};\n\t"
+      "mov.b64 m, {%5, %5};\n\t"
+      "add.rn.f32x2 x, x, k;\n\t"
+      "mul.rn.f32x2 x, x, m;\n\t"
+      "mov.b64 {%0, %1}, x;\n\t}"
+      : "=f"(r0), "=f"(r1)
+      : "r"(a0), "r"(a1), "f"(c), "f"(s));
+}
+
 __device__ __forceinline__ float sigmoidf_acc(float v) { return 1.0f / (1.0f + expf(-v)); }
 
 // SiLU(g) * u, the gated activation of the expert FFN

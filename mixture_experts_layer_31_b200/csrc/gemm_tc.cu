@@ -234,13 +234,17 @@ __device__ __forceinline__ uint4 widen8(const uint2 w, float scale) {
       o[2 * h + 1] = __byte_perm(__float_as_uint(f[2]), __float_as_uint(f[3]), 0x7632);
     }
   } else {
+    // int4: the subtraction and the scaling run on element pairs with the paired
+    // fp32 instructions (the same roundings as one element at a time); fewer
+    // instructions where the widening, not the tensor core, sets the pace
     const uint32_t lo = (w.x & 0x0F0F0F0Fu) ^ 0x08080808u;         // even elements, q + 8
     const uint32_t hi = ((w.x >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;  // odd elements
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float q0 = __uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7440u | j)) - 8388616.0f;
-      const float q1 = __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7440u | j)) - 8388616.0f;
-      o[j] = pack_bf16x2(q0 * scale, q1 * scale);
+      float v0, v1;
+      add_mul_f32x2(__byte_perm(lo, 0x4B000000u, 0x7440u | j), __byte_perm(hi, 0x4B000000u, 0x7440u | j),
+                    -8388616.0f, scale, v0, v1);
+      o[j] = pack_bf16x2(v0, v1);
     }
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
