@@ -12,15 +12,18 @@
 //            both against one token tile, so TMEM lane i holds both projections
 //            of output row i:  h[pos, i] = SiLU(s_g D0[i, pos]) * (s_u D1[i, pos])
 //   down:    1 or 2 M tiles of 128 W_down rows;  Yp[pair, r] = w_pair * s_d * D[r, pos]
+//            (Yp in fp32, or bf16 when the launch asks for it: large bf16 batches)
 // Storage: bf16 weights go straight from TMA into the 128-byte-swizzled
 // K-major layout the tensor core reads; int8 rows (one scale per row and
 // expert -- Kimi-Linear LiteRT-LM details, quantization bullet) are widened
 // exactly to bf16 by dequant warps and scaled in the epilogue; int4 block-32
 // (Qwen3 card, Available Artifacts table) is widened to q*s in bf16.
 //
-// Roles in a persistent CTA (one per SM), all walking one list of units:
-//   warp 0 lane 0   TMA producer: bf16 weight tiles and token boxes into one
-//                   stage ring; quantised weights: raw tiles into their own ring
+// Roles in a persistent CTA (one per SM), all walking one list of units that
+// warp 0 lane 0 claims from a per-launch counter and publishes, decoded, through
+// a small shared-memory queue:
+//   warp 0 lane 0   scheduler and TMA producer: bf16 weight tiles and token boxes
+//                   into one stage ring; quantised weights: raw tiles into their own ring
 //   warp 1          TMEM allocator; lane 0 issues tcgen05.mma, commits stages
 //   warp 2 lane 0   quantised weights only: TMA producer of the token boxes
 //   warps 4..11     epilogue (two 4-warp groups): tcgen05.ld -> activation / scales -> global
