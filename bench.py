@@ -177,28 +177,31 @@ def touched_experts(idx: np.ndarray, E: int) -> int:
     return int(np.unique(idx[(idx >= 0) & (idx < E)]).size)
 
 
-def algorithmic(prob, idx: np.ndarray):
-    """Per-launch algorithmic bytes / flops of the kernels, and the layer totals.
+def algorithmic(prob, idx: np.ndarray, path: str = "gemm"):
+    """Per-launch algorithmic bytes / flops of the dominant kernels, and the layer totals.
 
-    gate/up: per touched expert, the gate and up weight (+scale) bytes; plus x
-    read and h written.  down: per touched expert its down weight (+scale)
-    bytes; plus h read and the per-pair outputs written.  Flops count only the
-    routed work: 6*H*I per (token, slot) pair and 2*H*E for the router.
+    Only what the method itself must move counts (the scope table's unit): per
+    launch, the touched experts' weight (+ scale) bytes, x read once (gate/up) and
+    y written once (down).  The design's own intermediates -- the token rows
+    gathered in expert order (written and read back), h between the projections
+    and the per-pair outputs -- are reported apart as traffic_overhead.  Flops
+    count only the routed work: 6*H*I per (token, slot) pair and 2*H*E for the
+    router.
     """
     E, H, I, T, k = prob.E, prob.H, prob.I, prob.T, prob.k
     ut = touched_experts(idx, E)
     P = T * k
     xb = 2 if prob.xfmt == "bf16" else 4
     hb = 4 if prob.wfmt == "f32" else 2
+    ypb = 2 if (path == "gemm" and prob.xfmt == "bf16" and T >= 2048) else 4  # per-pair outputs: bf16 rows at T >= 2048
     per_mat = lambda W, S: W.nbytes // E + (0 if S is None else S.nbytes // E)
     gate_up_per_expert = per_mat(prob.W_gate, prob.s_gate) + per_mat(prob.W_up, prob.s_up)
     down_per_expert = per_mat(prob.W_down, prob.s_down)
-    bytes_ = {
-        "gemv_gateup": ut * gate_up_per_expert + T * H * xb + P * I * hb,
-        "gemm_gateup": ut * gate_up_per_expert + P * H * 2 + P * I * 2,
-        "gemv_down": ut * down_per_expert + P * I * hb + P * H * 4,
-        "gemm_down": ut * down_per_expert + P * I * 2 + P * H * 4,
-    }
+    gathered = 2 * P * H * 2 if path == "gemm" else 0  # rows gathered in expert order: written, then read
+    bytes_ = {"gemm_gateup": ut * gate_up_per_expert + T * H * xb, "gemv_gateup": ut * gate_up_per_expert + T * H * xb,
+              "gemm_down": ut * down_per_expert + T * H * xb, "gemv_down": ut * down_per_expert + T * H * xb}
+    overhead = {"gemm_gateup": gathered + P * I * hb, "gemv_gateup": P * I * hb,
+                "gemm_down": P * I * hb + P * H * ypb, "gemv_down": P * I * hb + P * H * ypb}
     flops = {"gemm_gateup": 4.0 * P * H * I, "gemm_down": 2.0 * P * H * I, "gemv_gateup": 4.0 * P * H * I,
              "gemv_down": 2.0 * P * H * I}
     layer_bytes = ut * (gate_up_per_expert + down_per_expert) + prob.W_r.nbytes + 2 * T * H * xb
@@ -210,14 +213,16 @@ def algorithmic(prob, idx: np.ndarray):
         layer_bytes += sh_up + sh_down
         layer_flops += 6.0 * T * H * prob.I_s
         # on the tensor-core path the shared expert's units run inside the routed launches
-        bytes_["gemm_gateup"] += sh_up + T * H * 2 + T * prob.I_s * 2
-        bytes_["gemm_down"] += sh_down + T * prob.I_s * 2 + T * H * 4
+        bytes_["gemm_gateup"] += sh_up
+        bytes_["gemm_down"] += sh_down
+        overhead["gemm_gateup"] += T * prob.I_s * 2
+        overhead["gemm_down"] += T * prob.I_s * 2 + T * H * 4
         flops["gemm_gateup"] += 4.0 * T * H * prob.I_s
         flops["gemm_down"] += 2.0 * T * H * prob.I_s
     if prob.residual is not None:
         layer_bytes += T * H * xb
     return dict(touched=ut, per_expert_gate_up=gate_up_per_expert, per_expert_down=down_per_expert, bytes=bytes_,
-                flops=flops, layer_bytes=layer_bytes, layer_flops=layer_flops)
+                overhead=overhead, flops=flops, layer_bytes=layer_bytes, layer_flops=layer_flops)
 
 
 def load_peaks():
@@ -260,17 +265,18 @@ def cpu_threads() -> int:
 
 def oracle_step(orc, tokens):
     """The oracle's pass over some tokens: route, experts, combine (and, for a block
-    workload, the shared expert and the residual)."""
+    workload, the shared expert and the residual).  Returns (y, idx, w, margin)."""
     p = orc.prob
     if p.I_s or p.residual is not None:
-        idx, w, _ = orc.route(tokens)
-        return orc.block(tokens, idx, w)
-    return orc.forward(tokens)[0]
+        idx, w, margin = orc.route(tokens)
+        return orc.block(tokens, idx, w), idx, w, margin
+    return orc.forward(tokens)
 
 
-def time_oracle(prob, budget_s: float, max_tokens=None):
+def time_oracle(prob, budget_s: float, max_tokens=None, seed: int = 0):
     """Time the fp64 oracle (route + experts + combine) on a seeded token sample
-    sized to roughly `budget_s` seconds of work; returns (tokens/s, threads, sample text)."""
+    sized to roughly `budget_s` seconds of work on all host cores.  Returns
+    (tokens/s, threads, sample text, tokens, (y, idx, w, margin))."""
     import oracle
     cores = cpu_threads()
     orc = oracle.Oracle(prob, nthreads=cores)
@@ -279,17 +285,38 @@ def time_oracle(prob, budget_s: float, max_tokens=None):
     per_token = max(time.perf_counter() - t0, 1e-6)  # one token, one thread
     n = int(budget_s * cores / per_token)
     n = max(1, min(n, prob.T if max_tokens is None else min(prob.T, max_tokens)))
-    rng = np.random.default_rng(0)
+    rng = np.random.default_rng(seed)
     toks = np.sort(rng.choice(prob.T, n, replace=False))
     t0 = time.perf_counter()
-    oracle_step(orc, toks)
+    out = oracle_step(orc, toks)
     dt = time.perf_counter() - t0
-    return n / dt, cores, "%d of %d tokens (seeded), route + experts + combine in fp64" % (n, prob.T)
+    return n / dt, cores, "%d of %d tokens (seeded), route + experts + combine in fp64" % (n, prob.T), toks, out
+
+
+def parity_record(prob, toks, ref, y_gpu, idx_gpu):
+    """The GPU's result on the oracle's sample tokens (taken outside the timed
+    region): indices against the oracle's where its k-th/(k+1)-th key margin
+    exceeds 1e-4, near-ties at or below it, and the relative L2 error of y over
+    the sample tokens whose expert sets agree (all of them, unless a near-tie
+    went the other way), with the worst single token."""
+    y_ref, idx_ref, _, margin = ref
+    gi = idx_gpu[toks]
+    same = (np.sort(gi, 1) == np.sort(idx_ref, 1)).all(1)
+    clear = margin > 1e-4
+    yg = y_gpu[toks].astype(np.float64)
+    d, r = yg[same] - y_ref[same], y_ref[same]
+    per = np.linalg.norm(d, axis=1) / np.maximum(np.linalg.norm(r, axis=1), 1e-300)
+    return {"sample_tokens": int(len(toks)), "clear_margin_tokens": int(clear.sum()),
+            "index_match_clear": int((same & clear).sum()), "near_ties": int((~clear).sum()),
+            "near_ties_same_experts": int((same & ~clear).sum()),
+            "rel_l2": float(np.linalg.norm(d) / max(np.linalg.norm(r), 1e-300)) if same.any() else None,
+            "worst_token_rel_l2": float(per.max()) if same.any() else None,
+            "rel_l2_bar": 1e-5 if (prob.xfmt == "f32" and prob.wfmt == "f32") else 5e-3}
 
 
 # ----------------------------------------------------------------------------- arms
 
-def config_block(prob, cid, extra=None):
+def config_block(prob, extra=None):
     c = {"workload": prob.cfg["workload"], "T": prob.T, "H": prob.H, "E": prob.E, "k": prob.k, "I": prob.I,
          "experts": prob.wfmt, "activations": prob.xfmt, "router": prob.router, "act": prob.act,
          "active_experts": int(prob.mask.sum()) if prob.mask is not None else prob.E,
@@ -332,10 +359,9 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_block(prob, args.config, {"sample_tokens_per_step": n,
-                                                        "block": ({"shared_I": prob.I_s,
-                                                                   "residual": prob.residual is not None}
-                                                                  if args.block else None)}),
+            "config": config_block(prob, {"sample_tokens_per_step": n,
+                                          "block": ({"shared_I": prob.I_s, "residual": prob.residual is not None}
+                                                    if args.block else None)}),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": "%d of %d tokens per step (seeded), route + experts + combine in fp64"
                                        % (n, prob.T)},
@@ -344,17 +370,37 @@ def run_reference(args):
     return 0
 
 
-def run_ours(args):
+def roofline(prob, acc, kern, stages, path_used):
+    """The dominant kernel's roofline: its algorithmic bytes and flops per launch over
+    its average launch time inside the timed steps, bound by its arithmetic
+    intensity against the measured ridge point; both fractions reported."""
+    peaks, peak_src = load_peaks()
+    of = "of measured" if peak_src == "measured" else "of fallback"
+    launches_k, total_k = stages.get(kern, (0, 0.0))
+    avg_ms = total_k / max(launches_k, 1)
+    kbytes, kflops = acc["bytes"][kern], acc["flops"][kern]
+    gbs = kbytes / (avg_ms * 1e-3) / 1e9
+    tfs = kflops / (avg_ms * 1e-3) / 1e12
+    t_hbm = kbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = kflops / (peaks["bf16_tflops"] * 1e12)
+    hbm_frac, tc_frac = gbs / peaks["hbm_gbs"], tfs / peaks["bf16_tflops"]
+    if t_hbm >= t_tc or path_used == "gemv":
+        roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": hbm_frac}
+    else:
+        roof = {"bound": "tensor", "achieved": tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": tc_frac}
+    roof.update({"kernel": kern, "avg_launch_ms": avg_ms, "algorithmic_bytes_per_launch": kbytes,
+                 "algorithmic_flops_per_launch": kflops, "traffic_overhead": acc["overhead"][kern],
+                 "hbm_frac": hbm_frac, "tensor_frac": tc_frac,
+                 "peak_source": "MEASURED_PEAKS.json hbm_gbs / bf16_tflops (burst), %s" % of})
+    roof["traffic"] = known_traffic(kern, prob.cfg["workload"])
+    return roof
+
+
+def measure(args, moe, prob, dev, local, world, headline: bool):
+    """Time one workload: warm-up, the device-resident timed steps (the dominant
+    kernel bracketed by events), the end-to-end steps (pinned host x in, y out),
+    and an untimed pass with every launch timed.  Returns (line fields, y, idx)."""
     import torch
-    rank, world, local = dist_env()
-    torch.cuda.set_device(local)
-    dist_init("nccl")
-    import mixture_experts_layer_31_b200 as moe
-    dev = torch.device("cuda", local)
-    if args.block:  # the whole MoE block: a shared expert of the routed size, and the residual
-        args.overrides.setdefault("shared", synth.config(args.config, **args.overrides)["I"])
-        args.overrides.setdefault("residual", True)
-    prob = synth.make_problem(args.config, replica=rank, **args.overrides)
     path = {"auto": moe.MOE_PATH_AUTO, "gemv": moe.MOE_PATH_GEMV, "gemm": moe.MOE_PATH_GEMM}[args.path]
     layer = moe.MoELayer(H=prob.H, I=prob.I, E=prob.E, k=prob.k, router=prob.router, scale=prob.scale,
                          wfmt=prob.wfmt, xfmt=prob.xfmt, W_r=prob.W_r, b=prob.b, expert_mask=prob.mask,
@@ -362,6 +408,8 @@ def run_ours(args):
                          s_up=prob.s_up, s_down=prob.s_down, path=path, device=dev, act=prob.act,
                          I_s=prob.I_s, Ws_gate=prob.Ws_gate, Ws_up=prob.Ws_up, Ws_down=prob.Ws_down,
                          ss_gate=prob.ss_gate, ss_up=prob.ss_up, ss_down=prob.ss_down)
+    block = headline and args.block
+    stats = headline and args.stats
     if prob.xfmt == "bf16":
         x_host = torch.from_numpy(prob.x.view(np.int16)).view(torch.bfloat16)
     else:
@@ -373,8 +421,7 @@ def run_ours(args):
     y = torch.empty((T, prob.H), dtype=layer.x_dtype, device=dev)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    counts = torch.zeros(prob.E, dtype=torch.uint64, device=dev) if args.stats else None
-
+    counts = torch.zeros(prob.E, dtype=torch.uint64, device=dev) if stats else None
     res_host = None
     if prob.residual is not None:
         res_host = torch.from_numpy(prob.residual.view(np.int16)).view(torch.bfloat16) if prob.xfmt == "bf16" \
@@ -383,13 +430,13 @@ def run_ours(args):
 
     def step(xin, yout, rin=None):
         rin = res if rin is None else rin
-        if not args.block and counts is None:  # the layer in one call (moe_layer_forward)
+        if not block and counts is None:  # the layer in one call (moe_layer_forward)
             layer.layer(xin, out=(yout, idx, w))
             return
         layer.route(xin, out=(idx, w))
         if counts is not None:  # routing-frequency recording (calibration runs)
             layer.expert_counts(idx, counts)
-        if args.block:
+        if block:
             layer.block(xin, idx, w, residual=rin, y=yout)
         else:
             layer.forward(xin, idx, w, y=yout)
@@ -398,7 +445,6 @@ def run_ours(args):
         step(x, y)
     torch.cuda.synchronize(dev)
     idx_np = idx.cpu().numpy()
-    acc = algorithmic(prob, idx_np)
     # which kernels the step runs (one untimed step with every launch timed)
     moe.moe_stage_times()
     moe.moe_stage_timing(True)
@@ -406,6 +452,7 @@ def run_ours(args):
     moe.moe_stage_timing(False)
     path_used = "gemm" if "gemm_gateup" in moe.moe_stage_times() else "gemv"
     kern = DOMINANT[path_used]
+    acc = algorithmic(prob, idx_np, path_used)
 
     # ---- device-resident timed region; events around the dominant kernel only
     # (two event records per timed launch; timing every launch would add about
@@ -432,6 +479,8 @@ def run_ours(args):
     step_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
     step_ms = max_over_ranks(step_ms, dev)
     value = world * T / (step_ms * 1e-3)
+    y_np = (y.view(torch.int16).cpu().numpy().view(np.uint16) if y.dtype == torch.bfloat16 else y.cpu().numpy())
+    idx_np = idx.cpu().numpy()
 
     # ---- end to end: pinned host x in, pinned host y out, copies inside each timed step
     xh = x_host.pin_memory()
@@ -470,53 +519,87 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     moe.moe_stage_timing(False)
     breakdown = moe.moe_stage_times()
+    peaks, _ = load_peaks()
 
-    # ---- roofline of the dominant kernel: bound by its arithmetic intensity
-    # (algorithmic flops per algorithmic byte) against the measured ridge point
-    peaks, peak_src = load_peaks()
-    of = "of measured" if peak_src == "measured" else "of fallback"
-    launches_k, total_k = stages.get(kern, (0, 0.0))
-    avg_ms = total_k / max(launches_k, 1)
-    kbytes, kflops = acc["bytes"][kern], acc["flops"][kern]
-    gbs = kbytes / (avg_ms * 1e-3) / 1e9
-    tfs = kflops / (avg_ms * 1e-3) / 1e12
-    t_hbm = kbytes / (peaks["hbm_gbs"] * 1e9)
-    t_tc = kflops / (peaks["bf16_tflops"] * 1e12)
-    hbm_frac, tc_frac = gbs / peaks["hbm_gbs"], tfs / peaks["bf16_tflops"]
-    if t_hbm >= t_tc or path_used == "gemv":
-        roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": hbm_frac}
-    else:
-        roof = {"bound": "tensor", "achieved": tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": tc_frac}
-    roof.update({"kernel": kern, "avg_launch_ms": avg_ms, "algorithmic_bytes_per_launch": kbytes,
-                 "algorithmic_flops_per_launch": kflops,
-                 "hbm_frac": hbm_frac, "tensor_frac": tc_frac,
-                 "peak_source": "MEASURED_PEAKS.json hbm_gbs / bf16_tflops (burst), %s" % of})
-    roof["traffic"] = known_traffic(kern, prob.cfg["workload"])
+    fields = {
+        "value": value, "ms_per_step": step_ms,
+        "dtype": "bf16" if prob.xfmt == "bf16" else "f32",
+        "config": config_block(prob, {"path": path_used, "touched_experts": acc["touched"],
+                                      "overrides": (args.overrides or None) if headline else None,
+                                      "routing_counts": bool(stats),
+                                      "block": ({"shared_I": prob.I_s, "residual": prob.residual is not None}
+                                                if block else None)}),
+        "roofline": roofline(prob, acc, kern, stages, path_used),
+        "layer": {"algorithmic_bytes": acc["layer_bytes"], "algorithmic_flops": acc["layer_flops"],
+                  "hbm_frac_of_step": acc["layer_bytes"] / (step_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                  "tensor_frac_of_step": acc["layer_flops"] / (step_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                  "kernels_ms": {n: round(t / max(c, 1), 5) for n, (c, t) in breakdown.items()},
+                  "kernels_ms_source": "separate pass after the timed region, every launch timed"},
+        "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": int(x.numel() * x.element_size())
+                                      + (0 if res is None else int(res.numel() * res.element_size())),
+                "d2h_bytes_per_step": int(y.numel() * y.element_size())},
+        "gpu_launches": int(launches),
+        "clocks": clocks.summary(),
+    }
+    del layer, x, y, idx, w, flush, xd, xh, yh
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    return fields, y_np, idx_np
 
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16" if prob.xfmt == "bf16" else "f32", "data": "synthetic",
-            "config": config_block(prob, args.config, {"path": path_used, "touched_experts": acc["touched"],
-                                                        "overrides": args.overrides or None,
-                                                        "routing_counts": bool(args.stats),
-                                                        "block": ({"shared_I": prob.I_s,
-                                                                   "residual": prob.residual is not None}
-                                                                  if args.block else None)}),
-            "roofline": roof,
-            "layer": {"algorithmic_bytes": acc["layer_bytes"], "algorithmic_flops": acc["layer_flops"],
-                      "hbm_frac_of_step": acc["layer_bytes"] / (step_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                      "kernels_ms": {n: round(t / max(c, 1), 5) for n, (c, t) in breakdown.items()},
-                      "kernels_ms_source": "separate pass after the timed region, every launch timed"},
-            "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT,
-                    "h2d_bytes_per_step": int(x.numel() * x.element_size())
-                                          + (0 if res is None else int(res.numel() * res.element_size())),
-                    "d2h_bytes_per_step": int(y.numel() * y.element_size())},
-            "gpu_launches": int(launches),
-            "clocks": clocks.summary(),
+
+def y_as_f64(prob, y_np):
+    if prob.xfmt == "bf16":
+        return synth.bf16_bits_to_f32(y_np).astype(np.float64)
+    return y_np.astype(np.float64)
+
+
+# the prefill-sized workloads timed beside the decode headline in the default run
+PER_CONFIG = (3, 4, 5)
+
+
+def run_ours(args):
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dist_init("nccl")
+    import mixture_experts_layer_31_b200 as moe
+    dev = torch.device("cuda", local)
+    if args.block:  # the whole MoE block: a shared expert of the routed size, and the residual
+        args.overrides.setdefault("shared", synth.config(args.config, **args.overrides)["I"])
+        args.overrides.setdefault("residual", True)
+    prob = synth.make_problem(args.config, replica=rank, **args.overrides)
+    fields, y_np, idx_np = measure(args, moe, prob, dev, local, world, headline=True)
+    line = {"metric": METRIC, "value": fields["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": fields["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": fields["dtype"], "data": "synthetic",
+            "config": fields["config"], "roofline": fields["roofline"], "layer": fields["layer"],
+            "e2e": fields["e2e"], "gpu_launches": fields["gpu_launches"], "clocks": fields["clocks"],
             "gpu": gpu_context(local)}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, sample = time_oracle(prob, budget_s=args.cpu_budget)
+    cpu_here = rank == 0 and world == 1 and not args.no_cpu_baseline
+    if cpu_here:
+        v, cores, sample, toks, ref = time_oracle(prob, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+        if not args.block:
+            line["parity"] = parity_record(prob, toks, ref, y_as_f64(prob, y_np), idx_np)
+    del prob
+    # the prefill-sized workloads, each measured the same way (one GPU; the metric's
+    # tensor-core half), with the oracle timed and compared on a bounded sample
+    if args.per_config and world == 1:
+        per = {}
+        for cid in PER_CONFIG:
+            p = synth.make_problem(cid)
+            f, yc, ic = measure(args, moe, p, dev, local, world, headline=False)
+            ent = {"tokens_per_s": f["value"], "ms_per_step": f["ms_per_step"], "dtype": f["dtype"],
+                   "config": f["config"], "roofline": f["roofline"], "layer": f["layer"], "e2e": f["e2e"],
+                   "gpu_launches": f["gpu_launches"], "clocks": f["clocks"]}
+            if cpu_here:
+                v, cores, sample, toks, ref = time_oracle(p, budget_s=args.cpu_budget_per_config, seed=cid)
+                ent["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+                ent["parity"] = parity_record(p, toks, ref, y_as_f64(p, yc), ic)
+            per[p.cfg["workload"]] = ent
+            del p, yc, ic
+        line["per_config"] = per
     if rank == 0:
         print(json.dumps(line), flush=True)
     barrier()
@@ -531,11 +614,16 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=2, choices=sorted(synth.CONFIGS))
+    ap.add_argument("--config", type=int, default=None, choices=sorted(synth.CONFIGS),
+                    help="the workload of the headline line (default 2, the Kimi decode batch)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--path", default="auto", choices=["auto", "gemv", "gemm"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--cpu-budget-per-config", type=float, default=8.0,
+                    help="seconds of oracle work for each per_config workload's cpu_baseline and parity sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time the headline workload only (the default run also times the prefill workloads)")
     ap.add_argument("--block", action="store_true",
                     help="time the whole MoE block: routed experts + a shared expert of the routed size + residual")
     ap.add_argument("--stats", action="store_true",
@@ -547,6 +635,11 @@ def main(argv=None):
     for kv in args.set:
         k_, v_ = kv.split("=", 1)
         args.overrides[k_] = int(v_) if v_.lstrip("-").isdigit() else v_
+    # the default invocation: the decode headline plus the prefill workloads
+    args.per_config = (args.config is None and not args.no_per_config and not args.block and not args.stats
+                       and not args.overrides and args.path == "auto")
+    if args.config is None:
+        args.config = 2
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

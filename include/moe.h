@@ -6,9 +6,9 @@
  *            top k chosen on score + bias, weights = the chosen SCORES
  *            renormalised and multiplied by a scale (2.446 for Kimi-Linear) --
  *            Kimi-Linear-48B-A3B LiteRT-LM details page, Conversion notes,
- *            mixture-of-experts bullet; CMF code specialist page, step 1 ("the
- *            sigmoid MoE router with its selection bias").  Or softmax, top k,
- *            renormalise (Qwen3-30B-A3B LiteRT-LM card, Conversion Notes).
+ *            mixture-of-experts bullet; the CMF code specialist page, step 1,
+ *            names the same sigmoid router and its selection bias.  Or softmax,
+ *            top k, renormalise (Qwen3-30B-A3B LiteRT-LM card, Conversion Notes).
  *   experts  only the k routed experts run for a token; each is a SiLU-gated
  *            FFN  o = W_down (SiLU(W_gate x) * (W_up x))  (Qwen3 card,
  *            Conversion Notes; the moe op's activation 'silu').
@@ -141,6 +141,22 @@ MOE_API moe_status moe_route(const moe_desc* d, const void* x, int32_t T, int32_
                      void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * The router logits l = W_r x that moe_route ranks: logits [T, E] fp32
+ * (row-major, 4-byte aligned, caller-owned; every expert, masked ones too --
+ * the mask acts on the keys, not on the logits).  Computed by the same kernels
+ * moe_route runs for this T, with the partial sums added in the same fixed
+ * order, so the values are exactly the ones moe_route (and moe_layer_forward)
+ * form their keys from: sigmoid(l) + b, or l itself for the softmax router
+ * (the router step of the Kimi-Linear LiteRT-LM details page, Conversion notes,
+ * and of the Qwen3-30B-A3B LiteRT-LM card, Conversion Notes).  For callers that
+ * need the logits themselves (auxiliary router losses, calibration) and for
+ * checking the routing against an exact reference.  Workspace as for
+ * moe_route; asynchronous on `stream`; errors as for moe_route.
+ */
+MOE_API moe_status moe_route_logits(const moe_desc* d, const void* x, int32_t T, float* logits, void* workspace,
+                                    size_t ws_bytes, cudaStream_t stream);
+
+/*
  * Experts + combine under a given routing (from moe_route or the caller):
  * y [T, H] in x's dtype, y[t] = sum_j topk_w[t, j] * FFN_{topk_idx[t, j]}(x[t])
  * summed in slot order in fp32, rounded once.  Slots whose index is outside
@@ -160,11 +176,16 @@ MOE_API moe_status moe_forward(const moe_desc* d, const void* x, int32_t T, cons
  * Scratch comes from one static device array of MOE_NOALLOC_SCRATCH_BYTES
  * that this library holds on every GPU that loads it, until the process
  * exits.  Inputs and outputs are still the caller's, exactly as for
- * moe_forward, and the result is the same as moe_forward's.  Problems whose
- * scratch (moe_workspace_size) exceeds the array -- roughly decode-sized
- * batches fit -- are rejected with MOE_ERR_WORKSPACE and a message; nothing is
- * launched then.  No cudaMalloc/cudaFree or other allocating call is made
- * (leave moe_stage_timing off: the timing itself creates CUDA events).
+ * moe_forward, and the result is bit for bit moe_forward's (the same kernels
+ * on the same data).  The forward pass alone needs less than
+ * moe_workspace_size reports (that size also covers moe_route's logits and
+ * its split router weights): sorted pairs, per-expert counts, the activations
+ * between the projections and the per-pair outputs, about
+ * T * k * (4 + 2 I + 6 H) bytes with bf16 activations -- some 115 tokens at
+ * H = 2304, I = 2048, k = 8.  Larger problems are rejected with
+ * MOE_ERR_WORKSPACE and a message naming both sizes; nothing is launched then.
+ * No cudaMalloc/cudaFree or other allocating call is made (leave
+ * moe_stage_timing off: the timing itself creates CUDA events).
  *
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
@@ -196,7 +217,7 @@ MOE_API moe_status moe_layer_forward(const moe_desc* d, const void* x, int32_t T
  *   y[t] = sum_j w[t,j] FFN_{idx[t,j]}(x[t])  +  FFN_shared(x[t])  +  residual[t]
  *
  * The shared expert is one more gated FFN applied to every token with weight 1
- * ("256-routed + 1-shared expert FFN" -- Kimi-Linear APEX quantization page;
+ * (the Kimi-Linear APEX quantization page lists 256 routed experts and one shared one;
  * the shared expert runs beside the moe op -- Kimi-Linear LiteRT-LM details
  * page, Conversion notes).  It uses the routed experts' activation (d->act) and
  * activation dtype; its own intermediate size I and storage format.  The

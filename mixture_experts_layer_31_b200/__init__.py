@@ -36,12 +36,26 @@ ACT = {"silu": MOE_ACT_SILU, "gelu_tanh": MOE_ACT_GELU_TANH}
 XFMT = {"f32": MOE_X_F32, "bf16": MOE_X_BF16}
 ROUTER = {"sigmoid": MOE_ROUTER_SIGMOID_BIAS, "softmax": MOE_ROUTER_SOFTMAX}
 
-EXPORTS = ("moe_workspace_size", "moe_route", "moe_forward", "moe_layer_forward", "moe_forward_noalloc",
+EXPORTS = ("moe_workspace_size", "moe_route", "moe_route_logits", "moe_forward", "moe_layer_forward", "moe_forward_noalloc",
            "moe_block_workspace_size",
            "moe_forward_block", "moe_expert_counts",
            "moe_cover_set", "moe_selftest_bounded_wait", "moe_last_error", "moe_device_flags", "moe_launch_count",
            "moe_stage_timing", "moe_stage_times", "moe_stage_timing_only")
-MOE_NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def _header_scratch_bytes() -> int:
+    """MOE_NOALLOC_SCRATCH_BYTES as include/moe.h defines it (the one definition;
+    the library is compiled from the same header)."""
+    import re
+    hdr = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
+    with open(hdr) as f:
+        m = re.search(r"#define\s+MOE_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", f.read())
+    if m is None:
+        raise ImportError("MOE_NOALLOC_SCRATCH_BYTES not found in %s" % hdr)
+    return int(m.group(1)) << int(m.group(2))
+
+
+MOE_NOALLOC_SCRATCH_BYTES = _header_scratch_bytes()
 
 
 class MoeError(RuntimeError):
@@ -81,6 +95,7 @@ def _load() -> ctypes.CDLL:
     lib.moe_workspace_size.argtypes = [D, i32, ctypes.POINTER(sz)]
     lib.moe_route.argtypes = [D, vp, i32, vp, vp, vp, sz, vp]
     lib.moe_forward.argtypes = [D, vp, i32, vp, vp, vp, vp, sz, vp]
+    lib.moe_route_logits.argtypes = [D, vp, i32, vp, vp, sz, vp]
     lib.moe_forward_noalloc.argtypes = [D, vp, i32, vp, vp, vp, vp]
     lib.moe_layer_forward.argtypes = [D, vp, i32, vp, vp, vp, vp, sz, vp]
     SH = ctypes.POINTER(moe_shared_expert)
@@ -98,7 +113,7 @@ def _load() -> ctypes.CDLL:
     lib.moe_stage_timing.argtypes = [i32]
     lib.moe_stage_times.argtypes = [ctypes.POINTER(moe_stage_time), i32, ctypes.POINTER(i32)]
     lib.moe_stage_timing_only.argtypes = [ctypes.c_char_p]
-    for f in ("moe_workspace_size", "moe_route", "moe_forward", "moe_layer_forward", "moe_forward_noalloc",
+    for f in ("moe_workspace_size", "moe_route", "moe_route_logits", "moe_forward", "moe_layer_forward", "moe_forward_noalloc",
               "moe_block_workspace_size",
               "moe_forward_block", "moe_expert_counts",
               "moe_cover_set", "moe_device_flags", "moe_stage_timing", "moe_stage_times", "moe_stage_timing_only"):
@@ -133,6 +148,12 @@ def moe_workspace_size(desc: moe_desc, T: int) -> int:
 def moe_route(desc: moe_desc, x: int, T: int, topk_idx: int, topk_w: int, workspace: int, ws_bytes: int,
               stream: int = 0) -> None:
     _check(lib().moe_route(ctypes.byref(desc), x, int(T), topk_idx, topk_w, workspace, int(ws_bytes), stream))
+
+
+def moe_route_logits(desc: moe_desc, x: int, T: int, logits: int, workspace: int, ws_bytes: int,
+                     stream: int = 0) -> None:
+    """logits [T, E] fp32: the router logits exactly as moe_route ranks them."""
+    _check(lib().moe_route_logits(ctypes.byref(desc), x, int(T), logits, workspace, int(ws_bytes), stream))
 
 
 def moe_forward(desc: moe_desc, x: int, T: int, topk_idx: int, topk_w: int, y: int, workspace: int,
@@ -303,6 +324,15 @@ class MoELayer:
         ws = self.workspace(T)
         moe_route(self.desc, x.data_ptr(), T, idx.data_ptr(), w.data_ptr(), ws.data_ptr(), ws.numel(), self._stream())
         return idx, w
+
+    def route_logits(self, x, out=None):
+        """The router logits [T, E] fp32 that route() ranks (moe_route_logits)."""
+        T = x.shape[0]
+        logits = out if out is not None else self.torch.empty((T, self.desc.E), dtype=self.torch.float32,
+                                                                device=self.device)
+        ws = self.workspace(T)
+        moe_route_logits(self.desc, x.data_ptr(), T, logits.data_ptr(), ws.data_ptr(), ws.numel(), self._stream())
+        return logits
 
     def forward(self, x, idx, w, y=None):
         T = x.shape[0]

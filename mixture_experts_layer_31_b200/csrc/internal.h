@@ -8,11 +8,13 @@
 
 namespace moe {
 
-// Programmatic dependent launch: every kernel of this library may start while
+// Programmatic dependent launch, opt-in (MOE_PDL=1 in the environment; plain
+// stream ordering otherwise): every kernel of this library may then start while
 // the kernel before it on the stream is finishing (its CTAs take SMs as they free
 // up and run their prologue); each waits (griddepcontrol.wait) before it reads
-// anything an earlier launch wrote, so results do not change.  MOE_PDL=0 in the
-// environment turns it off (plain stream ordering).
+// or writes anything an earlier launch touches, and only then lets the next
+// launch start, so results do not change.  Without the attribute the wait and
+// the trigger are no-ops.
 bool pdl_enabled();
 
 // Launch one kernel on stream s and report the launch status.
@@ -81,7 +83,15 @@ struct Workspace {
   size_t total;
 };
 
-Workspace carve_workspace(const moe_desc& d, int32_t T, void* base);
+// forward_only: the layout of a forward pass given its routing, without the
+// router-only regions (logits and w3 are then unusable)
+Workspace carve_workspace(const moe_desc& d, int32_t T, void* base, bool forward_only = false);
+// bytes of that forward-only layout
+size_t forward_scratch_bytes(const moe_desc& d, int32_t T);
+// moe_forward on a workspace of the full (forward_only = false) or the
+// forward-only layout
+moe_status forward_impl(const moe_desc* d, const void* x, int32_t T, const int32_t* topk_idx, const float* topk_w,
+                        void* y, void* workspace, size_t ws_bytes, cudaStream_t stream, bool forward_only);
 
 // set the calling thread's moe_last_error() message and return `code`
 moe_status report_error(moe_status code, const char* message);
@@ -95,6 +105,9 @@ cudaError_t launch_router_logits(const moe_desc& d, const void* x, int T, float*
                                  cudaStream_t s);
 cudaError_t launch_router_topk(const moe_desc& d, const float* partial, int S, int T, int32_t* idx,
                                float* w, uint32_t* flags, cudaStream_t s);
+// logits [T, E] = the S partials [S, T, E] summed in split order (as the top-k does)
+cudaError_t launch_logits_sum(const float* partial, int S, int T, int E, float* logits, int num_sms,
+                              cudaStream_t s);
 bool small_sort_ok(int P, int E);
 cudaError_t launch_small_sort(const int32_t* idx, int P, int E, int chunk, int32_t* counts, int32_t* offsets,
                               int32_t* touched, int32_t* group_base, int32_t* tile_base, int32_t* meta,

@@ -78,10 +78,12 @@ static moe_status device_state(DeviceState** out) {
 static std::atomic<uint64_t> g_launches{0};
 static std::atomic<int> g_timing{0};
 
+// Programmatic dependent launch is opt-in: MOE_PDL=1 in the environment (read
+// once per process).  Plain stream ordering is the default.
 bool pdl_enabled() {
   static const bool on = [] {
     const char* v = getenv("MOE_PDL");
-    return !(v != nullptr && v[0] == '0');
+    return v != nullptr && v[0] == '1';
   }();
   return on;
 }
@@ -207,7 +209,9 @@ static size_t up256(size_t v) { return (v + 255) / 256 * 256; }
 
 constexpr int kRegions = 13;
 
-static void layout(const moe_desc& d, int32_t T, size_t off[kRegions], size_t* total) {
+// forward_only: the router-only regions (partial logits, split router weights)
+// take no space -- the layout of a forward pass that is given its routing
+static void layout(const moe_desc& d, int32_t T, size_t off[kRegions], size_t* total, bool forward_only = false) {
   const size_t P = (size_t)T * d.k, E = d.E;
   const size_t S_simt = router_splits(T), S_tc = d.xfmt == MOE_X_BF16 ? router_tc_splits(T, d.H) : 0;
   size_t S = S_simt > S_tc ? S_simt : S_tc;
@@ -216,9 +220,9 @@ static void layout(const moe_desc& d, int32_t T, size_t off[kRegions], size_t* t
   const size_t NC = (P + kPairChunk - 1) / kPairChunk;
   const size_t hbytes = d.wfmt == MOE_W_F32 ? 4 : 2;
   const size_t xs_bytes = (d.xfmt == MOE_X_BF16 && d.wfmt != MOE_W_F32) ? P * d.H * 2 : 0;
-  const size_t sizes[kRegions] = {S * T * E * 4, (NC ? NC : 1) * E * 4, E * 4, (E + 1) * 4, (E + 1) * 4, 16 * 4,
-                                  P * 4, P * d.I * hbytes, P * d.H * 4, xs_bytes, (E + 1) * 4, (E + 1) * 4,
-                                  w3_bytes};
+  const size_t sizes[kRegions] = {forward_only ? 0 : S * T * E * 4, (NC ? NC : 1) * E * 4, E * 4, (E + 1) * 4,
+                                  (E + 1) * 4, 16 * 4, P * 4, P * d.I * hbytes, P * d.H * 4, xs_bytes, (E + 1) * 4,
+                                  (E + 1) * 4, forward_only ? 0 : w3_bytes};
   size_t o = 0;
   for (int i = 0; i < kRegions; ++i) {
     off[i] = o;
@@ -227,9 +231,9 @@ static void layout(const moe_desc& d, int32_t T, size_t off[kRegions], size_t* t
   *total = o;
 }
 
-Workspace carve_workspace(const moe_desc& d, int32_t T, void* base) {
+Workspace carve_workspace(const moe_desc& d, int32_t T, void* base, bool forward_only) {
   size_t off[kRegions], total;
-  layout(d, T, off, &total);
+  layout(d, T, off, &total, forward_only);
   char* b = static_cast<char*>(base);
   Workspace w;
   w.logits = reinterpret_cast<float*>(b + off[0]);
@@ -249,9 +253,15 @@ Workspace carve_workspace(const moe_desc& d, int32_t T, void* base) {
   return w;
 }
 
-static moe_status check_ws(const moe_desc& d, int32_t T, void* ws, size_t ws_bytes) {
+size_t forward_scratch_bytes(const moe_desc& d, int32_t T) {
   size_t off[kRegions], need;
-  layout(d, T, off, &need);
+  layout(d, T, off, &need, true);
+  return need;
+}
+
+static moe_status check_ws(const moe_desc& d, int32_t T, void* ws, size_t ws_bytes, bool forward_only = false) {
+  size_t off[kRegions], need;
+  layout(d, T, off, &need, forward_only);
   if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL (need %zu bytes)", need);
   if (!aligned(ws, 256)) return fail(MOE_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   if (ws_bytes < need) return fail(MOE_ERR_WORKSPACE, "workspace too small: %zu bytes given, %zu needed", ws_bytes, need);
@@ -275,6 +285,9 @@ extern "C" moe_status moe_workspace_size(const moe_desc* d, int32_t T, size_t* b
   return MOE_OK;
 }
 
+static moe_status route_partial_logits(const moe_desc* d, const void* x, int32_t T, const Workspace& ws,
+                                       DeviceState* dev, cudaStream_t stream, int* S_out);
+
 extern "C" moe_status moe_route(const moe_desc* d, const void* x, int32_t T, int32_t* topk_idx, float* topk_w,
                                 void* workspace, size_t ws_bytes, cudaStream_t stream) {
   g_err.clear();
@@ -289,6 +302,35 @@ extern "C" moe_status moe_route(const moe_desc* d, const void* x, int32_t T, int
   DeviceState* dev = nullptr;
   if ((st = device_state(&dev)) != MOE_OK) return st;
   const Workspace ws = carve_workspace(*d, T, workspace);
+  int S = 0;
+  if ((st = route_partial_logits(d, x, T, ws, dev, stream, &S)) != MOE_OK) return st;
+  MOE_LAUNCH("router_topk", stream, launch_router_topk(*d, ws.logits, S, T, topk_idx, topk_w, dev->flags, stream));
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_route_logits(const moe_desc* d, const void* x, int32_t T, float* logits, void* workspace,
+                                       size_t ws_bytes, cudaStream_t stream) {
+  g_err.clear();
+  moe_status st = validate_desc(d);
+  if (st != MOE_OK) return st;
+  if ((st = validate_T(T, d->k)) != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!x || !aligned(x, 16)) return fail(MOE_ERR_INVALID_ARG, "x must be a non-NULL 16-byte aligned device pointer");
+  if (!logits || !aligned(logits, 4)) return fail(MOE_ERR_INVALID_ARG, "logits must be non-NULL, 4-byte aligned");
+  if ((st = check_ws(*d, T, workspace, ws_bytes)) != MOE_OK) return st;
+  DeviceState* dev = nullptr;
+  if ((st = device_state(&dev)) != MOE_OK) return st;
+  const Workspace ws = carve_workspace(*d, T, workspace);
+  int S = 0;
+  if ((st = route_partial_logits(d, x, T, ws, dev, stream, &S)) != MOE_OK) return st;
+  MOE_LAUNCH("router_logits_sum", stream, launch_logits_sum(ws.logits, S, T, d->E, logits, dev->num_sms, stream));
+  return MOE_OK;
+}
+
+// the router's partial logits [S, T, E] into ws.logits, by the kernels moe_route
+// uses for this T; *S_out = S
+static moe_status route_partial_logits(const moe_desc* d, const void* x, int32_t T, const Workspace& ws,
+                                       DeviceState* dev, cudaStream_t stream, int* S_out) {
   int S;
   if (decode_route_ok(*d, T)) {
     // decode-sized batch: fp32 logits from fp32 W_r in one launch, every H-split
@@ -305,7 +347,7 @@ extern "C" moe_status moe_route(const moe_desc* d, const void* x, int32_t T, int
     S = router_splits(T);
     MOE_LAUNCH("router_logits", stream, launch_router_logits(*d, x, T, ws.logits, S, stream));
   }
-  MOE_LAUNCH("router_topk", stream, launch_router_topk(*d, ws.logits, S, T, topk_idx, topk_w, dev->flags, stream));
+  *S_out = S;
   return MOE_OK;
 }
 
@@ -356,24 +398,32 @@ static moe_status check_io(const void* x, const void* y, const int32_t* topk_idx
 static const char* kNoTensorCores =
     "tensor-core path needs bf16 activations, bf16/int8/int4 weights and H, I multiples of 128";
 
-extern "C" moe_status moe_forward(const moe_desc* d, const void* x, int32_t T, const int32_t* topk_idx,
-                                  const float* topk_w, void* y, void* workspace, size_t ws_bytes,
-                                  cudaStream_t stream) {
+// moe_forward's work; forward_only carves the workspace without the
+// router-only regions (the layout forward_scratch_bytes sizes)
+moe_status moe::forward_impl(const moe_desc* d, const void* x, int32_t T, const int32_t* topk_idx,
+                             const float* topk_w, void* y, void* workspace, size_t ws_bytes, cudaStream_t stream,
+                             bool forward_only) {
   g_err.clear();
   moe_status st = validate_desc(d);
   if (st != MOE_OK) return st;
   if ((st = validate_T(T, d->k)) != MOE_OK) return st;
   if (T == 0) return MOE_OK;
   if ((st = check_io(x, y, topk_idx, topk_w)) != MOE_OK) return st;
-  if ((st = check_ws(*d, T, workspace, ws_bytes)) != MOE_OK) return st;
+  if ((st = check_ws(*d, T, workspace, ws_bytes, forward_only)) != MOE_OK) return st;
   const int path = choose_path(*d, T);
   if (path == MOE_PATH_GEMM && !gemm_capable(*d)) return fail(MOE_ERR_UNSUPPORTED, "%s", kNoTensorCores);
   DeviceState* dev = nullptr;
   if ((st = device_state(&dev)) != MOE_OK) return st;
-  const Workspace ws = carve_workspace(*d, T, workspace);
+  const Workspace ws = carve_workspace(*d, T, workspace, forward_only);
   if ((st = run_routed(d, x, T, topk_idx, topk_w, ws, path, dev, stream)) != MOE_OK) return st;
   MOE_LAUNCH("combine", stream, launch_combine(*d, topk_idx, T, ws.yp, yp_bf16(*d, T, path), y, stream));
   return MOE_OK;
+}
+
+extern "C" moe_status moe_forward(const moe_desc* d, const void* x, int32_t T, const int32_t* topk_idx,
+                                  const float* topk_w, void* y, void* workspace, size_t ws_bytes,
+                                  cudaStream_t stream) {
+  return forward_impl(d, x, T, topk_idx, topk_w, y, workspace, ws_bytes, stream, false);
 }
 
 // ------------------------------------------------------------------ route and forward in one call

@@ -60,10 +60,13 @@ cudaError_t scratch_address(void** out, int* dev_out) {
 
 extern "C" moe_status moe_forward_noalloc(const moe_desc* d, const void* x, int32_t T, const int32_t* topk_idx,
                                           const float* topk_w, void* y, cudaStream_t stream) {
-  size_t need = 0;
-  moe_status st = moe_workspace_size(d, T, &need);  // validates the descriptor and T
+  size_t full = 0;
+  moe_status st = moe_workspace_size(d, T, &full);  // validates the descriptor and T
   if (st != MOE_OK) return st;
   if (T == 0) return MOE_OK;
+  // the forward pass alone: the routing is given, so the router's regions of
+  // moe_workspace_size's layout are left out
+  const size_t need = moe::forward_scratch_bytes(*d, T);
   if (need > (size_t)MOE_NOALLOC_SCRATCH_BYTES) {
     char msg[256];
     snprintf(msg, sizeof(msg),
@@ -81,5 +84,5 @@ extern "C" moe_status moe_forward_noalloc(const moe_desc* d, const void* x, int3
              cudaGetErrorString(e));
     return moe::report_error(MOE_ERR_CUDA, msg);
   }
-  return moe_forward(d, x, T, topk_idx, topk_w, y, scratch, (size_t)MOE_NOALLOC_SCRATCH_BYTES, stream);
+  return moe::forward_impl(d, x, T, topk_idx, topk_w, y, scratch, (size_t)MOE_NOALLOC_SCRATCH_BYTES, stream, true);
 }

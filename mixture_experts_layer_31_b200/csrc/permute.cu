@@ -1,7 +1,7 @@
 // Expert-sorted order of the (token, slot) pairs: histogram, scan, stable
-// counting-sort scatter.  "only the 8 routed experts are computed for each
-// token" (Qwen3-30B-A3B LiteRT-LM card, Conversion Notes): grouping the pairs
-// by expert lets each expert's weights be streamed once for all its tokens.
+// counting-sort scatter.  A token runs only through its routed experts
+// (Qwen3-30B-A3B LiteRT-LM card, Conversion Notes): grouping the pairs by
+// expert lets each expert's weights be streamed once for all its tokens.
 //
 // Pair p = t * k + slot.  The pairs are cut into chunks of kPairChunk; every
 // kernel walks a chunk in pair order, so the result is a deterministic, stable

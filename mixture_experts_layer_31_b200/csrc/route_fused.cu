@@ -1,11 +1,10 @@
 // Router and expert sort for decode-sized batches, fused to two launches.
 //
-// "the router in plain ops (sigmoid scores, the top 8 chosen on the scores plus
-// the correction bias, weights renormalized and scaled by 2.446)" (Kimi-Linear
-// LiteRT-LM details page, Conversion notes); the sort groups the (token, slot)
-// pairs by expert so that each expert's weights stream once ("only the 8
-// routed experts are computed for each token" -- Qwen3-30B-A3B LiteRT-LM card,
-// Conversion Notes).
+// The router is the Kimi-Linear one: sigmoid scores, top 8 on score plus
+// correction bias, chosen scores renormalised and scaled by 2.446 (Kimi-Linear
+// LiteRT-LM details page, Conversion notes).  The sort groups the (token, slot)
+// pairs by expert so that each expert's weights stream once; a token runs only
+// through its routed experts (Qwen3-30B-A3B LiteRT-LM card, Conversion Notes).
 //
 //   decode_logits_kernel  fp32 partial logits [S, T, E] straight from fp32
 //                         W_r (S from 1 to 8: about 128 CTAs, and a slice of

@@ -1,12 +1,12 @@
 // Router of the routed-MoE layer: fp32 logits, sigmoid+selection-bias or
 // softmax keys, warp-shuffle top-k, renormalised weights times the scale.
 //
-// "the router in plain ops (sigmoid scores, the top 8 chosen on the scores
-// plus the correction bias, weights renormalized and scaled by 2.446)" --
-// Kimi-Linear LiteRT-LM details page, Conversion notes; "The router, its
-// softmax, the top 8 and their renormalization" -- Qwen3-30B-A3B LiteRT-LM
-// card, Conversion Notes.  Masked experts are never selectable (CMF page,
-// Defrag step: runtime expert mask).
+// Kimi-Linear: sigmoid scores pick the top 8 after the correction bias is
+// added; the chosen scores are renormalised and multiplied by 2.446
+// (Kimi-Linear LiteRT-LM details page, Conversion notes).  Qwen3: softmax, top
+// 8, renormalisation, all as plain graph ops (Qwen3-30B-A3B LiteRT-LM card,
+// Conversion Notes).  Masked experts are never selectable (CMF page, Defrag
+// step: runtime expert mask).
 //
 // Two kernels:
 //   router_logits_kernel  tiled SIMT fp32 GEMM, partial[s][t][e] over S splits
@@ -136,7 +136,30 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
   route_dev::warp_topk<PER_LANE, S>(partial, T, t, E, k, router, bias, mask, scale, idx, wout, flags);
 }
 
+// logits[t][e] = the S partial sums added in split order from 0.f: the same
+// additions, in the same order, as the top-k kernels perform before ranking
+__global__ void __launch_bounds__(256) logits_sum_kernel(const float* __restrict__ partial, int S, int T, int E,
+                                                         float* __restrict__ logits) {
+  pdl_wait();
+  pdl_trigger();
+  const size_t n = (size_t)T * E;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    float sum = 0.f;
+    for (int s = 0; s < S; ++s) sum += partial[(size_t)s * n + i];
+    logits[i] = sum;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_logits_sum(const float* partial, int S, int T, int E, float* logits, int num_sms,
+                              cudaStream_t s) {
+  const size_t n = (size_t)T * E;
+  int blocks = (int)((n + 255) / 256);
+  if (blocks > num_sms * 8) blocks = num_sms * 8;
+  if (blocks < 1) blocks = 1;
+  return launch_k(logits_sum_kernel, dim3(blocks), dim3(256), 0, s, partial, S, T, E, logits);
+}
 
 cudaError_t launch_router_logits(const moe_desc& d, const void* x, int T, float* partial, int S,
                                  cudaStream_t s) {

@@ -12,22 +12,21 @@
  *   1. logits   l_e = sum_h W_r[e,h] x[t,h]                   for every expert e
  *   2. keys     sigmoid router: s_e = 1/(1+exp(-l_e)), key_e = s_e + b_e
  *               softmax router: key_e = exp(l_e - m) / sum_{a active} exp(l_a - m)
- *      "sigmoid scores, the top 8 chosen on the scores plus the correction
- *       bias, weights renormalized and scaled by 2.446" -- Kimi-Linear LiteRT-LM
- *       details page, Conversion notes, mixture-of-experts bullet; "the sigmoid
- *       MoE router with its selection bias" -- CMF code specialist page, How it
- *       was made step 1.  "The router, its softmax, the top 8 and their
- *       renormalization are ordinary ops" -- Qwen3-30B-A3B LiteRT-LM card,
- *       Conversion Notes.
+ *      Kimi-Linear: top 8 on sigmoid score plus correction bias, the chosen
+ *       scores renormalised and scaled by 2.446 -- Kimi-Linear LiteRT-LM
+ *       details page, Conversion notes, mixture-of-experts bullet; the CMF code
+ *       specialist page (How it was made, step 1) names the same sigmoid router
+ *       and selection bias.  Qwen3: softmax, top 8 and renormalisation as
+ *       plain ops -- Qwen3-30B-A3B LiteRT-LM card, Conversion Notes.
  *   3. top-k    sort the ACTIVE experts by (key descending, index ascending) and
- *               keep the first k; masked experts are never selectable ("Runtime
- *               semantics equal the runtime expert mask" -- CMF page, Defrag).
+ *               keep the first k; masked experts are never selectable (the CMF
+ *               page's Defrag step equates the sliced file with a runtime mask).
  *   4. weights  w_j = r_j / sum_{selected} r * scale, with r = s (sigmoid scores,
  *               WITHOUT the bias, which only selects) or r = p (softmax).
  *   5. experts  for each selected e: g = W_gate[e] x, u = W_up[e] x,
  *               a = act(g) * u  (gated), o = W_down[e] a; act = SiLU,
  *               g * sigmoid(g), or GELU in its tanh form.
- *               "only the 8 routed experts are computed for each token" --
+ *               a token runs only through its 8 routed experts --
  *               Qwen3 card, Conversion Notes; activation 'silu' -- same card and
  *               the Kimi details page (moe op with SiLU); the moe op's other
  *               activation, 'gelu_tanh', is named by the same two passages (the
@@ -309,7 +308,7 @@ int oracle_forward(const oracle_layer* L, const void* x, int64_t t0, int64_t t1,
  * The whole MoE block for tokens [t0, t1) under a given routing:
  *   y[t] = sum_j w_j o_{idx_j}(x_t)  +  shared(x_t)  +  residual[t]
  * The routed sum is oracle_combine's; shared(x) is one more gated FFN with
- * weight 1 over every token ("256-routed + 1-shared expert FFN" -- Kimi-Linear
+ * weight 1 over every token (256 routed experts plus one shared one -- Kimi-Linear
  * APEX quantization page, intro; the shared expert runs beside the moe op --
  * Kimi-Linear LiteRT-LM details page, Conversion notes, mixture-of-experts
  * bullet), described by S as a one-expert layer (S->E == 1, same H and

@@ -17,13 +17,13 @@
  * thread count.  Normals use the Box-Muller transform on consecutive pairs.
  *
  * Storage encoders (the pages' formats):
- *  - int8 per output channel: "routed experts int8 per channel (one scale per
- *    output row and expert)", "symmetric, min-max" -- Kimi-Linear LiteRT-LM
- *    details page, Conversion notes, quantization bullet.  s = max|w|/127,
+ *  - int8 per output channel: the routed experts carry one symmetric min-max
+ *    scale per output row and expert -- Kimi-Linear LiteRT-LM details page,
+ *    Conversion notes, quantization bullet.  s = max|w|/127,
  *    q = clamp(round_half_away(w/s), -127, 127); an all-zero row gets s = 1.
- *  - int4 block 32: "experts int4 blockwise (block 32, fp32 scales)" and
- *    "Int4 block scales below 2^-14 are raised to 2^-14" -- Qwen3-30B-A3B
- *    LiteRT-LM model card, Available Artifacts table and Conversion Notes.
+ *  - int4 block 32: blockwise int4 experts, 32 columns per fp32 scale, with
+ *    scales under 2^-14 lifted to 2^-14 -- Qwen3-30B-A3B LiteRT-LM model card,
+ *    Available Artifacts table and Conversion Notes.
  *    Blocks run along the reduction axis; s = max(max|w|/7, 2^-14),
  *    q = clamp(round_half_away(w/s), -8, 7), two's-complement nibbles, the
  *    low nibble holding the even column.

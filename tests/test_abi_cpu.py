@@ -91,8 +91,15 @@ def test_route_and_forward_validate_before_launch():
     with pytest.raises(moe.MoeError) as ei:  # negative T
         moe.moe_forward(d, 1 << 20, -1, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 30)
     assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+    with pytest.raises(moe.MoeError) as ei:  # NULL logits
+        moe.moe_route_logits(d, 1 << 20, 16, None, 1 << 20, 1 << 30)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+    with pytest.raises(moe.MoeError) as ei:  # workspace too small for the router's partial logits
+        moe.moe_route_logits(d, 1 << 20, 16, 1 << 20, 1 << 20, 256)
+    assert ei.value.status == moe.MOE_ERR_WORKSPACE
     # T = 0 is a valid no-op that launches nothing
     n = moe.moe_launch_count()
+    moe.moe_route_logits(d, 1 << 20, 0, None, None, 0)
     moe.moe_route(d, 1 << 20, 0, 1 << 20, 1 << 20, None, 0)
     moe.moe_forward(d, 1 << 20, 0, 1 << 20, 1 << 20, 1 << 20, None, 0)
     assert moe.moe_launch_count() == n

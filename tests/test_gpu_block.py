@@ -8,7 +8,8 @@ import torch
 
 import mixture_experts_layer_31_b200 as moe
 import synth
-from gpu_util import judge, judge_block, layer_from_problem, x_to_device
+from gpu_util import (chunk_tokens, dense_cover_tokens, gpu_logits, judge, judge_block, layer_from_problem,
+                      unit_cover_tokens, x_to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -50,7 +51,7 @@ def test_block_small(name):
     cid, over = CASES[name]
     prob = synth.make_problem(cid, **over)
     layer, x, idx, w, res, y = _run_block(prob)
-    judge(prob, layer.forward(x, idx, w), idx, w)  # the routing itself
+    judge(prob, layer.forward(x, idx, w), idx, w, logits=gpu_logits(layer, x))  # the routing itself
     judge_block(prob, y, idx, w)
 
 
@@ -62,11 +63,16 @@ def test_block_decode_full_size():
     judge_block(prob, y, idx, w)
 
 
-def test_block_prefill_sampled():
+def test_block_prefill_every_unit():
+    """The int8 prefill widths with a shared expert of the routed size and a
+    residual: the checked tokens reach every routed (expert, token chunk) unit and
+    every unit of the shared expert, which runs as a dense problem (every token in
+    order) inside the same grouped-GEMM launches."""
     prob = synth.make_problem(3, T=2048, shared=2048, residual=True)
     _, _, idx, w, _, y = _run_block(prob)
-    rng = np.random.default_rng(5)
-    judge_block(prob, y, idx, w, tokens=np.unique(np.concatenate([[0, prob.T - 1], rng.choice(prob.T, 30)])))
+    routed, _ = unit_cover_tokens(idx.cpu().numpy(), prob.E, prob.T, prob.k)
+    dense = dense_cover_tokens(prob.T, chunk_tokens(prob.T, 1, 1))
+    judge_block(prob, y, idx, w, tokens=np.unique(np.concatenate([routed, dense])))
 
 
 @pytest.mark.parametrize("T", [300, 2100])

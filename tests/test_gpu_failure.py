@@ -10,7 +10,7 @@ import torch
 
 import mixture_experts_layer_31_b200 as moe
 import synth
-from gpu_util import judge, run
+from gpu_util import gpu_logits, judge, run
 
 pytestmark = pytest.mark.gpu
 
@@ -26,6 +26,6 @@ def test_bounded_wait_gives_up_and_the_context_stays_usable():
     assert flags & MOE_FLAG_TIMEOUT
     assert 1.0 < elapsed < 30.0
     prob = synth.make_problem(3, T=40, H=256, E=16, I=128)
-    _, _, y, idx, w = run(prob)
-    judge(prob, y, idx, w)
+    layer, x, y, idx, w = run(prob)
+    judge(prob, y, idx, w, logits=gpu_logits(layer, x))
     assert moe.moe_device_flags(clear=True) == 0

@@ -7,7 +7,7 @@ import torch
 
 import mixture_experts_layer_31_b200 as moe
 import synth
-from gpu_util import judge, layer_from_problem, x_to_device
+from gpu_util import gpu_logits, judge, layer_from_problem, x_to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -40,7 +40,7 @@ def test_layer_forward_matches_oracle_and_the_separate_steps(name):
     x = x_to_device(prob)
     y, idx, w = layer.layer(x)
     torch.cuda.synchronize()
-    judge(prob, y, idx, w)
+    judge(prob, y, idx, w, logits=gpu_logits(layer, x))
     # the separate entry points on the same input: same routing, same output, bit for bit
     i2, w2 = layer.route(x)
     y2 = layer.forward(x, i2, w2)
@@ -53,9 +53,10 @@ def test_layer_forward_matches_oracle_and_the_separate_steps(name):
 def test_layer_forward_full_decode_shape():
     prob = synth.make_problem(2)
     layer = layer_from_problem(prob)
-    y, idx, w = layer.layer(x_to_device(prob))
+    x = x_to_device(prob)
+    y, idx, w = layer.layer(x)
     torch.cuda.synchronize()
-    judge(prob, y, idx, w)
+    judge(prob, y, idx, w, logits=gpu_logits(layer, x))
 
 
 def test_decode_router_mask_equals_slice():
@@ -106,9 +107,10 @@ def test_layer_forward_edge_shapes(name):
     cid, over = EDGE[name]
     prob = synth.make_problem(cid, **over)
     layer = layer_from_problem(prob)
-    y, idx, w = layer.layer(x_to_device(prob))
+    x = x_to_device(prob)
+    y, idx, w = layer.layer(x)
     torch.cuda.synchronize()
-    judge(prob, y, idx, w)
+    judge(prob, y, idx, w, logits=gpu_logits(layer, x))
     if prob.mask is not None:
         assert prob.mask[idx.cpu().numpy()].all()
 
@@ -171,9 +173,9 @@ def test_layer_replays_from_a_cuda_graph(cid, over):
 
 
 def test_programmatic_launch_does_not_change_results(tmp_path):
-    """The same layer calls with programmatic dependent launch (the default) and
-    with plain stream ordering (MOE_PDL=0, read once per process, so in a child
-    process) give the same bits."""
+    """The same layer calls with programmatic dependent launch (opt-in, MOE_PDL=1,
+    read once per process, so in a child process) and with plain stream ordering
+    (the default) give the same bits."""
     import os
     import subprocess
     import sys
