@@ -45,11 +45,13 @@ __device__ __forceinline__ float sigmoidf_acc(float v) { return 1.0f / (1.0f + e
 // SiLU(g) * u, the gated activation of the expert FFN
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
-// The same with CUDA's fast intrinsics (a few ulp), for outputs rounded to bf16
-// afterwards.  The exponent argument is capped so 1 + e stays below 2^126, the
-// range where __fdividef is exact to its stated error.
-// tanh-form GELU of the gate times up.  (1 + tanh z) / 2 = 1 / (1 + exp(-2z)),
+// tanh-form GELU of the gate times up: the tanh approximation of GELU from
+// Hendrycks and Gimpel, "Gaussian Error Linear Units (GELUs)", 2016, whose
+// constants are sqrt(2/pi) and 0.044715.  (1 + tanh z) / 2 = 1 / (1 + exp(-2z)),
 // so gelu(g) = g / (1 + exp(-2z)) with z = sqrt(2/pi) (g + 0.044715 g^3).
+// The *_fast forms use CUDA's fast intrinsics (a few ulp), for outputs rounded
+// to bf16 afterwards; the exponent argument is capped so 1 + e stays below
+// 2^126, the range where __fdividef is exact to its stated error.
 __device__ __forceinline__ float gelu_tanh_z(float g) {
   return 0.7978845608028654f * fmaf(0.044715f * g, g * g, g);
 }
@@ -110,14 +112,21 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// A waiting thread is suspended in the barrier until the phase completes, or
+// for at most this long (the PTX suspend-time hint); it then resumes at once
+// when the phase completes.  Without the hint the hardware's own, shorter limit
+// applies, and waiting warps re-issue their wait loop often enough to take
+// issue slots from the warps doing the work.
+constexpr uint32_t kSuspendHintNs = 1000000u;  // 1 ms
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
@@ -137,7 +146,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1; i != 0; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if ((i & 7u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) return false;
   }
   return false;
 }
@@ -220,6 +229,19 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16: A is 128 rows (TMEM lanes) x 16
+// bf16 (8 columns of bf16 pairs, the lower K index in the low half) from TMEM
+// address a_tmem (lane 0)
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // arrive (once) on `bar` when every tcgen05 operation issued so far by this thread completes
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -240,6 +262,26 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 }
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 16 registers per thread -> 32 lanes x 16 consecutive 32-bit TMEM columns
+// (the warp's own lane quarter); complete after tmem_st_wait
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// 8 registers per thread -> 32 lanes x 8 consecutive 32-bit TMEM columns
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // make generic-proxy writes to shared memory visible to the async proxy (tensor core, TMA)
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }

@@ -1,7 +1,7 @@
 // Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
 //
-// "only the 8 routed experts are computed for each token" (Qwen3-30B-A3B
-// LiteRT-LM card, Conversion Notes): after the tokens are sorted by expert,
+// A token runs only through its 8 routed experts (Qwen3-30B-A3B LiteRT-LM
+// card, Conversion Notes): after the tokens are sorted by expert,
 // every expert e owns a contiguous run of m_e rows.  A unit of work is
 // (expert e, block of output rows, chunk of up to `chunk` of e's tokens),
 // computed swap-AB:  D[128 weight rows, N tokens] = A[128, K] * X_e[N, K]^T,
@@ -83,6 +83,7 @@ struct GemmArgs {
   int acc_stride;       // TMEM columns per M tile accumulator (power of two >= chunk)
   int nbuf;             // accumulator buffers (2: epilogue overlaps the next unit's MMAs)
   int tmem_cols;        // TMEM columns allocated
+  int a_col0;           // quantised, A in TMEM: first TMEM column of the widened A stages
   // router logits (MODE 2): dense [T, E] = x [T, H] . W3 [E, 3H]^T over S splits of the K steps
   int T;
   int S;
@@ -209,14 +210,6 @@ __device__ __forceinline__ void shfl_unit(Unit& t) {
   t.dense = __shfl_sync(0xFFFFFFFFu, t.dense ? 1 : 0, 0) != 0;
 }
 
-// Raw bytes of one 8-element chunk: 8 bytes of int8, or 4 bytes of packed int4
-// (in .x).
-template <int WF>
-__device__ __forceinline__ uint2 load_chunk(const uint8_t* raw_chunk) {
-  if constexpr (WF == MOE_W_INT8_ROW) return *reinterpret_cast<const uint2*>(raw_chunk);
-  return make_uint2(*reinterpret_cast<const uint32_t*>(raw_chunk), 0u);
-}
-
 // Widen one 8-element chunk of a raw quantised row to bf16.
 // int8: byte-permute (q + 128) into the low byte of the fp32 2^23 and subtract
 // 2^23 + 128 -> exact q; |q| <= 128 has <= 8 significant bits, so the top half
@@ -253,28 +246,34 @@ __device__ __forceinline__ uint4 widen8(const uint2 w, float scale) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-template <int MODE, int WF, int MT>
+// TA (quantised weights only): the widened A tiles live in TMEM and the MMA
+// reads A from there (tcgen05.mma [d], [a], b-desc) -- shared memory then
+// carries only the raw bytes and the token tiles; otherwise they live in a
+// shared-memory ring in the 128-byte swizzle.
+template <int MODE, int WF, int MT, int TA>
 struct Traits {
   static constexpr bool kQuant = WF != MOE_W_BF16;
+  static constexpr bool kTmemA = kQuant && TA != 0;
   // gate/up: MT = 2 (gate tile, up tile) over 128 output rows; down: MT tiles of 128 rows
   static constexpr int kRows = MODE == 0 ? kBM : kBM * MT;  // output rows per unit
   static constexpr int kRawTile = WF == MOE_W_INT8_ROW ? kBM * kBK : (WF == MOE_W_INT4_B32 ? kBM * kBK / 2 : 0);
-  static constexpr int kRawPitch = WF == MOE_W_INT8_ROW ? kBK : kBK / 2;  // bytes per raw row
+  static constexpr int kAcols = kTmemA ? MT * (kBK / 2) : 0;  // TMEM columns of one widened A stage
   static constexpr int kEpiWarps = 8;                     // two 4-warp groups
   static constexpr int kDequantWarps = kQuant ? 8 : 0;
   static constexpr int kDequant0 = 4 + kEpiWarps;         // first dequant warp
   static constexpr int kThreads = 32 * (4 + kEpiWarps + kDequantWarps);
   static constexpr int kGroupXchg = MODE == 0 ? 0 : 2 * 256 * 4;  // down: pair ids + weights per group
   static constexpr int kXchg = (2 * kGroupXchg + 1023) / 1024 * 1024;
+  static constexpr int kARing = kQuant && !kTmemA ? kAStages * MT * kTileBytes : 0;  // shared-memory A ring
 };
 
-template <int MODE, int WF, int MT>
-__global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
+template <int MODE, int WF, int MT, int TA>
+__global__ void __launch_bounds__(Traits<MODE, WF, MT, TA>::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
                    const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_w0d,
                    const __grid_constant__ CUtensorMap tm_w1d, const __grid_constant__ CUtensorMap tm_bd,
                    const GemmArgs a) {
-  using Tr = Traits<MODE, WF, MT>;
+  using Tr = Traits<MODE, WF, MT, TA>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_base + 1023u) & ~1023u) - raw_base);  // 1024-aligned
@@ -293,8 +292,8 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
   Unit* unit_tq = reinterpret_cast<Unit*>(unit_q + kUnitQ);  // [kUnitQ] the same units, decoded
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unit_tq + kUnitQ);
   float* xchg = reinterpret_cast<float*>(smem + kBarrierBytes);
-  uint8_t* a_ring = smem + kBarrierBytes + Tr::kXchg;  // quantised: kAStages x MT bf16 A tiles
-  uint8_t* stages = a_ring + (Tr::kQuant ? kAStages * MT * kTileBytes : 0);
+  uint8_t* a_ring = smem + kBarrierBytes + Tr::kXchg;  // quantised, A in shared memory: kAStages x MT bf16 A tiles
+  uint8_t* stages = a_ring + Tr::kARing;
   uint8_t* raw_ring = stages + a.raw_ring_off;  // quantised only
 
   const int w = warp_id(), lane = lane_id();
@@ -476,13 +475,18 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
           tc_fence_after();
           const uint32_t sb = stage0 + s * a.stage_bytes;
           const uint32_t sa = Tr::kQuant ? a_ring0 + ja * (MT * kTileBytes) : sb;
+          const uint32_t ta = tmem_base + (uint32_t)(a.a_col0 + ja * Tr::kAcols);  // TMEM A: lane 0 of the stage
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
             const uint64_t bdesc = umma_desc_sw128(sb + a.b_off + k * 32);
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-              umma_bf16(d + mt * a.acc_stride, umma_desc_sw128(sa + mt * kTileBytes + k * 32), bdesc, idesc,
-                        (kb | k) != 0);
+            for (int mt = 0; mt < MT; ++mt) {
+              if constexpr (Tr::kTmemA)  // A: 128 lanes x 8 columns of bf16 pairs per K = 16
+                umma_bf16_ts(d + mt * a.acc_stride, ta + mt * (kBK / 2) + k * 8, bdesc, idesc, (kb | k) != 0);
+              else
+                umma_bf16(d + mt * a.acc_stride, umma_desc_sw128(sa + mt * kTileBytes + k * 32), bdesc, idesc,
+                          (kb | k) != 0);
+            }
           }
           umma_commit(&empty[s]);
           if (Tr::kQuant) umma_commit(&a_empty[ja]);
@@ -630,13 +634,21 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
     }
   } else if (Tr::kQuant && w >= Tr::kDequant0) {
     // ------------------------------------------------------------------ dequantisation
-    // thread ct widens chunks (r, c8): r = ct/8 + kRowStep*j over the unit's MT*128
-    // weight rows, c8 = ct%8 -- 8 elements each
-    constexpr int kDT = 32 * (Tr::kDequantWarps > 0 ? Tr::kDequantWarps : 1);
-    constexpr int kRowStep = kDT / 8;
-    constexpr int kPer = MT * kBM / kRowStep;  // chunks per thread per K step
+    // One weight row per thread (two threads per row when the unit has 128 A rows):
+    // thread ct owns row r = ct % (MT*128) of the unit's A rows and the 8-element
+    // chunks [cg*kChunks, (cg+1)*kChunks) of it, cg = ct / (MT*128).  The raw tiles
+    // arrive in the TMA's 64-byte (int8) or 32-byte (int4) swizzle, so a warp's 32
+    // rows read their 16-byte pieces without bank conflicts, and the widened
+    // chunks go to the 128-byte-swizzled bf16 tile the same way.  An int4 row
+    // needs two block scales per K step (one per 32 columns), not one per chunk.
+    constexpr int kDT = 32 * (Tr::kDequantWarps > 0 ? Tr::kDequantWarps : 8);  // dequant threads
+    constexpr int kRowsA = MT * kBM;
+    constexpr int kChunks = 8 * kRowsA / kDT;  // chunks per thread per K step (8 or 4)
+    static_assert(kDT % kRowsA == 0 && kChunks >= 1 && kChunks <= 8, "dequant thread mapping");
     const int ct = threadIdx.x - 32 * Tr::kDequant0;
-    const int c8 = ct & 7, r0 = ct >> 3;
+    const int r = ct % kRowsA, cg = ct / kRowsA;
+    const int mt = r >> 7, rr = r & 127;
+    const int c0 = cg * kChunks;  // first chunk of this thread
     bool dead = false;
     uint32_t it = 0;
     int rs = 0;        // raw-ring slot of K step `it`
@@ -648,27 +660,22 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
       u = __shfl_sync(0xFFFFFFFFu, u, 0);
       if (u < 0) break;
       shfl_unit(t);
-      // int4: block scales of this thread's rows, one K step ahead
+      // int4: this row's block scales for the chunks of this thread, one K step ahead
       const ProbView pv = view_of(a, t);
-      const float* srow[kPer];
-      float sc_next[kPer];
-#pragma unroll
-      for (int j = 0; j < kPer; ++j) {
-        const int r = r0 + kRowStep * j;  // row within the unit's MT*128 A rows
-        const int mt = r >> 7, rr = r & 127;
-        const float* S = (MODE == 0 && mt == 1) ? pv.s1 : pv.s0;
-        int wr = MODE == 0 ? t.ib * kBM + rr : t.ib * Tr::kRows + mt * kBM + rr;
-        if (wr >= pv.R) wr = pv.R - 1;  // rows past a half block are computed but never stored
-        srow[j] = S + ((size_t)t.e * pv.R + wr) * (pv.K >> a.qsh);
-        sc_next[j] = WF == MOE_W_INT4_B32 ? __ldg(srow[j] + ((t.k0 * kBK + c8 * 8) >> a.qsh)) : 1.f;
+      const float* S = (MODE == 0 && mt == 1) ? pv.s1 : pv.s0;
+      int wr = MODE == 0 ? t.ib * kBM + rr : t.ib * Tr::kRows + mt * kBM + rr;
+      if (wr >= pv.R) wr = pv.R - 1;  // rows past a half block are computed but never stored
+      const float* srow = S + ((size_t)t.e * pv.R + wr) * (pv.K >> a.qsh);
+      float s_next[2] = {1.f, 1.f};  // scales of chunks c0 and c0 + kChunks - 1 (the two 32-column halves)
+      if (WF == MOE_W_INT4_B32) {
+        s_next[0] = __ldg(srow + ((t.k0 * kBK + c0 * 8) >> a.qsh));
+        s_next[1] = __ldg(srow + ((t.k0 * kBK + (c0 + kChunks - 1) * 8) >> a.qsh));
       }
       for (int kb = 0; kb < t.nk; ++kb, ++it) {
-        float sc[kPer];
-#pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-          sc[j] = sc_next[j];
-          if (WF == MOE_W_INT4_B32 && kb + 1 < t.nk)
-            sc_next[j] = __ldg(srow[j] + (((t.k0 + kb + 1) * kBK + c8 * 8) >> a.qsh));
+        const float s_lo = s_next[0], s_hi = s_next[1];
+        if (WF == MOE_W_INT4_B32 && kb + 1 < t.nk) {
+          s_next[0] = __ldg(srow + (((t.k0 + kb + 1) * kBK + c0 * 8) >> a.qsh));
+          s_next[1] = __ldg(srow + (((t.k0 + kb + 1) * kBK + (c0 + kChunks - 1) * 8) >> a.qsh));
         }
         const int s = rs;
         const uint32_t ph = rph;
@@ -676,24 +683,72 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT>::kThreads, 1)
         const int ja = it % kAStages;
         wait_or_die(&rfull[s], ph, dead, a.flags);
         wait_or_die(&a_empty[ja], ((it / kAStages) & 1u) ^ 1u, dead, a.flags);
+        if constexpr (Tr::kTmemA) dead = __any_sync(0xFFFFFFFFu, dead);  // tcgen05.st below is warp-collective
         if (!dead) {
-          const uint8_t* raw = raw_ring + (size_t)s * a.raw_stage_bytes;
-          uint8_t* A = a_ring + ja * (MT * kTileBytes);
-          // all loads first, then the independent widen+store chains
-          uint2 q[kPer];
+          const uint8_t* raw = raw_ring + (size_t)s * a.raw_stage_bytes + mt * Tr::kRawTile;
+          uint8_t* A = a_ring + ja * (MT * kTileBytes) + mt * kTileBytes + rr * 128;
+          // the row's raw bytes of this thread's chunks: 16-byte pieces, all loads first
+          uint32_t q[kChunks * (WF == MOE_W_INT8_ROW ? 2 : 1)];
+          if constexpr (WF == MOE_W_INT8_ROW) {
+            // 64-byte rows, piece p (chunks 2p, 2p+1) at (p ^ ((rr >> 1) & 3)) * 16
 #pragma unroll
-          for (int j = 0; j < kPer; ++j) {
-            const int r = r0 + kRowStep * j;
-            const int mt = r >> 7, rr = r & 127;
-            q[j] = load_chunk<WF>(raw + mt * Tr::kRawTile + rr * Tr::kRawPitch + c8 * (Tr::kRawPitch / 8));
-          }
+            for (int p = 0; p < kChunks / 2; ++p) {
+              const int pp = c0 / 2 + p;
+              const uint4 v = *reinterpret_cast<const uint4*>(raw + rr * 64 + ((pp ^ ((rr >> 1) & 3)) << 4));
+              q[4 * p] = v.x; q[4 * p + 1] = v.y; q[4 * p + 2] = v.z; q[4 * p + 3] = v.w;
+            }
+          } else {
+            // 32-byte rows, piece p (chunks 4p .. 4p+3) at (p ^ ((rr >> 2) & 1)) * 16
 #pragma unroll
-          for (int j = 0; j < kPer; ++j) {
-            const int r = r0 + kRowStep * j;
-            const int mt = r >> 7, rr = r & 127;
-            *reinterpret_cast<uint4*>(A + mt * kTileBytes + rr * 128 + ((c8 ^ (rr & 7)) << 4)) = widen8<WF>(q[j], sc[j]);
+            for (int p = 0; p < (kChunks + 3) / 4; ++p) {
+              const int pp = c0 / 4 + p;
+              const uint4 v = *reinterpret_cast<const uint4*>(raw + rr * 32 + ((pp ^ ((rr >> 2) & 1)) << 4));
+              q[4 * p] = v.x; q[4 * p + 1] = v.y; q[4 * p + 2] = v.z; q[4 * p + 3] = v.w;
+            }
           }
-          fence_proxy_async_smem();
+          if constexpr (Tr::kTmemA) {
+            // the row's widened chunks are 4 * kChunks consecutive bf16-pair columns of
+            // this thread's TMEM lane (lower K in the low half): one warp-wide store
+            // into the warp's lane quarter (warp w reaches lanes 32 (w % 4) .. + 31,
+            // and rr / 32 == w % 4 by the row mapping above)
+            tc_fence_after();  // after a_empty: the MMAs that read this stage are complete
+            uint32_t words[4 * kChunks];
+#pragma unroll
+            for (int j = 0; j < kChunks; ++j) {
+              const uint2 raw8 = WF == MOE_W_INT8_ROW ? make_uint2(q[2 * j], q[2 * j + 1]) : make_uint2(q[j], 0u);
+              const uint4 o = widen8<WF>(raw8, j * 2 < kChunks ? s_lo : s_hi);
+              words[4 * j] = o.x;
+              words[4 * j + 1] = o.y;
+              words[4 * j + 2] = o.z;
+              words[4 * j + 3] = o.w;
+            }
+            const uint32_t taddr = tmem_base + ((uint32_t)(rr & ~31) << 16) +
+                                   (uint32_t)(a.a_col0 + ja * Tr::kAcols + mt * (kBK / 2) + c0 * 4);
+#pragma unroll
+            for (int h = 0; h < kChunks / 4; ++h) {
+              uint32_t part[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) part[i] = words[16 * h + i];
+              tmem_st16(taddr + 16 * h, part);
+            }
+            if constexpr (kChunks % 4 != 0) {  // two chunks: 8 columns
+              uint32_t part[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) part[i] = words[4 * kChunks - 8 + i];
+              tmem_st8(taddr + 4 * kChunks - 8, part);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+          } else {
+#pragma unroll
+            for (int j = 0; j < kChunks; ++j) {
+              const int c = c0 + j;
+              const uint2 raw8 = WF == MOE_W_INT8_ROW ? make_uint2(q[2 * j], q[2 * j + 1]) : make_uint2(q[j], 0u);
+              const float sc = j * 2 < kChunks ? s_lo : s_hi;
+              *reinterpret_cast<uint4*>(A + ((c ^ (rr & 7)) << 4)) = widen8<WF>(raw8, sc);
+            }
+            fence_proxy_async_smem();
+          }
         }
         __syncwarp();
         if (lane == 0) {
@@ -749,8 +804,8 @@ cudaError_t weight_map(CUtensorMap* m, const void* W, int wfmt, int E, int R, in
   if (wfmt == MOE_W_BF16)
     return make_map(m, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, rows, kBK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
   if (wfmt == MOE_W_INT8_ROW)
-    return make_map(m, W, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, rows, kBK, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
-  return make_map(m, W, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, rows, kBK / 2, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
+    return make_map(m, W, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, rows, kBK, box_rows, CU_TENSOR_MAP_SWIZZLE_64B);
+  return make_map(m, W, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, rows, kBK / 2, box_rows, CU_TENSOR_MAP_SWIZZLE_32B);
 }
 
 uint32_t pow2_at_least(uint32_t v) {
@@ -765,24 +820,26 @@ struct Maps {
   CUtensorMap w0, w1, b, w0d, w1d, bd;
 };
 
-template <int MODE, int WF, int MT>
-cudaError_t launch_gemm(const Maps& m, GemmArgs a, int num_sms, cudaStream_t s) {
-  using Tr = Traits<MODE, WF, MT>;
-  // the dense problem's units: (row block of Tr::kRows, token chunk)
-  a.dense_units = a.Td > 0 ? ((a.Rd + Tr::kRows - 1) / Tr::kRows) * ((a.Td + a.chunkd - 1) / a.chunkd) : 0;
-  const int chunk_max = a.dense_units > 0 && a.chunkd > a.chunk ? a.chunkd : a.chunk;
+template <int MODE, int WF, int MT, int TA>
+cudaError_t launch_gemm(const Maps& m, GemmArgs a, int chunk_max, int num_sms, cudaStream_t s) {
+  using Tr = Traits<MODE, WF, MT, TA>;
   // stage: bf16 weights [A: MT x 16 KB][B]; quantised [B], with the raw tiles in a ring of
-  // their own after the main ring (their bf16 A lives in the A ring).  Token boxes are
-  // kBoxRows tall: B holds the chunk rounded up to whole boxes.  All sizes are multiples of
-  // 1024 (4 KB boxes, 16/8/4 KB tiles).
+  // their own after the main ring (their bf16 A lives in the A ring or in TMEM).  Token
+  // boxes are kBoxRows tall: B holds the chunk rounded up to whole boxes.  All sizes are
+  // multiples of 1024 (4 KB boxes, 16/8/4 KB tiles).
   const int b_rows = (chunk_max + kBoxRows - 1) / kBoxRows * kBoxRows;
   a.b_off = Tr::kQuant ? 0 : MT * kTileBytes;
   a.stage_bytes = a.b_off + b_rows * kBK * 2;
   a.raw_stage_bytes = MT * Tr::kRawTile;
+  // TMEM: nbuf accumulator sets of MT tiles, then (A in TMEM) kAStages widened A stages
   a.acc_stride = (int)pow2_at_least((uint32_t)chunk_max);
-  a.nbuf = 2 * MT * a.acc_stride <= 512 ? 2 : 1;
-  a.tmem_cols = a.nbuf * MT * a.acc_stride;
-  const int fixed = 1024 + kBarrierBytes + Tr::kXchg + (Tr::kQuant ? kAStages * MT * kTileBytes : 0);
+  const int acols = kAStages * Tr::kAcols;
+  a.nbuf = 2 * MT * a.acc_stride + acols <= 512 ? 2 : 1;
+  const int tcols = a.nbuf * MT * a.acc_stride + acols;
+  if (tcols > 512) return cudaErrorInvalidConfiguration;
+  a.tmem_cols = (int)pow2_at_least((uint32_t)tcols);
+  a.a_col0 = a.nbuf * MT * a.acc_stride;
+  const int fixed = 1024 + kBarrierBytes + Tr::kXchg + Tr::kARing;
   const int avail = kSmemLimit - fixed;
   if (Tr::kQuant) {
     // token ring: about 96 KB of boxes (L2-resident rows), 2..4 stages; the rest feeds the
@@ -801,10 +858,18 @@ cudaError_t launch_gemm(const Maps& m, GemmArgs a, int num_sms, cudaStream_t s) 
   if (a.NS < 2) return cudaErrorInvalidConfiguration;
   a.raw_ring_off = a.NS * a.stage_bytes;
   const size_t smem = (size_t)fixed + (size_t)a.NS * a.stage_bytes + (size_t)a.RS * a.raw_stage_bytes;
-  auto kern = gemm_tc_kernel<MODE, WF, MT>;
+  auto kern = gemm_tc_kernel<MODE, WF, MT, TA>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   return launch_k(kern, dim3(num_sms), dim3(Tr::kThreads), smem, s, m.w0, m.w1, m.b, m.w0d, m.w1d, m.bd, a);
+}
+
+// Quantised weights widen into TMEM when the accumulators leave room for the
+// widened A stages (chunks of at most 128 tokens); otherwise into shared memory.
+template <int MODE, int WF, int MT>
+cudaError_t launch_quant(const Maps& m, const GemmArgs& a, int chunk_max, int num_sms, cudaStream_t s) {
+  if (chunk_max <= 128) return launch_gemm<MODE, WF, MT, 1>(m, a, chunk_max, num_sms, s);
+  return launch_gemm<MODE, WF, MT, 0>(m, a, chunk_max, num_sms, s);
 }
 
 // gate/up always carries two M tiles (gate, up); down carries two 128-row tiles
@@ -813,17 +878,22 @@ cudaError_t launch_gemm(const Maps& m, GemmArgs a, int num_sms, cudaStream_t s) 
 // 16 KB tile per stage about 86%; at prefill sizes the token tile feeds 256
 // weight rows)
 template <int MODE>
-cudaError_t launch_by_format(int wfmt, const Maps& m, const GemmArgs& a, int num_sms, cudaStream_t s) {
+cudaError_t launch_by_format(int wfmt, const Maps& m, GemmArgs a, int num_sms, cudaStream_t s) {
   const bool two = MODE == 0 || a.R % (2 * kBM) == 0;  // down: the dense problem has the same R (= H)
+  // the dense problem's units: (row block of kRows, token chunk)
+  const int rows = MODE == 0 || !two ? kBM : 2 * kBM;
+  a.dense_units = a.Td > 0 ? ((a.Rd + rows - 1) / rows) * ((a.Td + a.chunkd - 1) / a.chunkd) : 0;
+  const int chunk_max = a.dense_units > 0 && a.chunkd > a.chunk ? a.chunkd : a.chunk;
   switch (wfmt) {
     case MOE_W_BF16:
-      return two ? launch_gemm<MODE, MOE_W_BF16, 2>(m, a, num_sms, s) : launch_gemm<MODE, MOE_W_BF16, 1>(m, a, num_sms, s);
+      return two ? launch_gemm<MODE, MOE_W_BF16, 2, 0>(m, a, chunk_max, num_sms, s)
+                 : launch_gemm<MODE, MOE_W_BF16, 1, 0>(m, a, chunk_max, num_sms, s);
     case MOE_W_INT8_ROW:
-      return two ? launch_gemm<MODE, MOE_W_INT8_ROW, 2>(m, a, num_sms, s)
-                 : launch_gemm<MODE, MOE_W_INT8_ROW, 1>(m, a, num_sms, s);
+      return two ? launch_quant<MODE, MOE_W_INT8_ROW, 2>(m, a, chunk_max, num_sms, s)
+                 : launch_quant<MODE, MOE_W_INT8_ROW, 1>(m, a, chunk_max, num_sms, s);
     default:
-      return two ? launch_gemm<MODE, MOE_W_INT4_B32, 2>(m, a, num_sms, s)
-                 : launch_gemm<MODE, MOE_W_INT4_B32, 1>(m, a, num_sms, s);
+      return two ? launch_quant<MODE, MOE_W_INT4_B32, 2>(m, a, chunk_max, num_sms, s)
+                 : launch_quant<MODE, MOE_W_INT4_B32, 1>(m, a, chunk_max, num_sms, s);
   }
 }
 
@@ -950,7 +1020,7 @@ cudaError_t launch_router_tc(const moe_desc& d, const void* x, int T, const void
   a.S = S;
   a.Hx = d.H;
   const Maps m{ma, ma, mb, ma, ma, mb};
-  return launch_gemm<2, MOE_W_BF16, 1>(m, a, num_sms, s);
+  return launch_gemm<2, MOE_W_BF16, 1, 0>(m, a, a.chunk, num_sms, s);
 }
 
 // gate/up tiles 128 output rows of I (a multiple of 64; a half block is computed
