@@ -84,6 +84,7 @@ struct GemmArgs {
   int nbuf;             // accumulator buffers (2: epilogue overlaps the next unit's MMAs)
   int tmem_cols;        // TMEM columns allocated
   int a_col0;           // quantised, A in TMEM: first TMEM column of the widened A stages
+  int a_stride;         // and the TMEM columns from one A stage to the next
   // router logits (MODE 2): dense [T, E] = x [T, H] . W3 [E, 3H]^T over S splits of the K steps
   int T;
   int S;
@@ -475,7 +476,7 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT, TA>::kThreads, 1)
           tc_fence_after();
           const uint32_t sb = stage0 + s * a.stage_bytes;
           const uint32_t sa = Tr::kQuant ? a_ring0 + ja * (MT * kTileBytes) : sb;
-          const uint32_t ta = tmem_base + (uint32_t)(a.a_col0 + ja * Tr::kAcols);  // TMEM A: lane 0 of the stage
+          const uint32_t ta = tmem_base + (uint32_t)(a.a_col0 + ja * a.a_stride);  // TMEM A: lane 0 of the stage
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
             const uint64_t bdesc = umma_desc_sw128(sb + a.b_off + k * 32);
@@ -681,14 +682,13 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT, TA>::kThreads, 1)
         const uint32_t ph = rph;
         if (++rs == a.RS) { rs = 0; rph ^= 1u; }
         const int ja = it % kAStages;
+        // the row's raw bytes of this thread's chunks (16-byte pieces) are loaded as soon
+        // as they have landed, before the wait for the A stage, so that the load latency
+        // overlaps that wait
         wait_or_die(&rfull[s], ph, dead, a.flags);
-        wait_or_die(&a_empty[ja], ((it / kAStages) & 1u) ^ 1u, dead, a.flags);
-        if constexpr (Tr::kTmemA) dead = __any_sync(0xFFFFFFFFu, dead);  // tcgen05.st below is warp-collective
+        uint32_t q[kChunks * (WF == MOE_W_INT8_ROW ? 2 : 1)];
         if (!dead) {
           const uint8_t* raw = raw_ring + (size_t)s * a.raw_stage_bytes + mt * Tr::kRawTile;
-          uint8_t* A = a_ring + ja * (MT * kTileBytes) + mt * kTileBytes + rr * 128;
-          // the row's raw bytes of this thread's chunks: 16-byte pieces, all loads first
-          uint32_t q[kChunks * (WF == MOE_W_INT8_ROW ? 2 : 1)];
           if constexpr (WF == MOE_W_INT8_ROW) {
             // 64-byte rows, piece p (chunks 2p, 2p+1) at (p ^ ((rr >> 1) & 3)) * 16
 #pragma unroll
@@ -706,6 +706,11 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT, TA>::kThreads, 1)
               q[4 * p] = v.x; q[4 * p + 1] = v.y; q[4 * p + 2] = v.z; q[4 * p + 3] = v.w;
             }
           }
+        }
+        wait_or_die(&a_empty[ja], ((it / kAStages) & 1u) ^ 1u, dead, a.flags);
+        if constexpr (Tr::kTmemA) dead = __any_sync(0xFFFFFFFFu, dead);  // tcgen05.st below is warp-collective
+        if (!dead) {
+          uint8_t* A = a_ring + ja * (MT * kTileBytes) + mt * kTileBytes + rr * 128;
           if constexpr (Tr::kTmemA) {
             // the row's widened chunks are 4 * kChunks consecutive bf16-pair columns of
             // this thread's TMEM lane (lower K in the low half): one warp-wide store
@@ -723,7 +728,7 @@ __global__ void __launch_bounds__(Traits<MODE, WF, MT, TA>::kThreads, 1)
               words[4 * j + 3] = o.w;
             }
             const uint32_t taddr = tmem_base + ((uint32_t)(rr & ~31) << 16) +
-                                   (uint32_t)(a.a_col0 + ja * Tr::kAcols + mt * (kBK / 2) + c0 * 4);
+                                   (uint32_t)(a.a_col0 + ja * a.a_stride + mt * (kBK / 2) + c0 * 4);
 #pragma unroll
             for (int h = 0; h < kChunks / 4; ++h) {
               uint32_t part[16];
@@ -831,14 +836,32 @@ cudaError_t launch_gemm(const Maps& m, GemmArgs a, int chunk_max, int num_sms, c
   a.b_off = Tr::kQuant ? 0 : MT * kTileBytes;
   a.stage_bytes = a.b_off + b_rows * kBK * 2;
   a.raw_stage_bytes = MT * Tr::kRawTile;
-  // TMEM: nbuf accumulator sets of MT tiles, then (A in TMEM) kAStages widened A stages
+  // TMEM.  Shared-memory A: nbuf accumulator sets of MT tiles.  A in TMEM, two
+  // layouts: "stacked" -- two accumulator sets, then the kAStages widened A stages --
+  // while that fits (chunks up to 64 tokens with two tiles); otherwise, two tiles of
+  // at most 192 tokens, "interleaved" -- one accumulator set, tile t at column 256 t
+  // and A stage j in the 64 columns after it (192 + 256 j) -- so every region starts
+  // on a multiple of 64 columns.
   a.acc_stride = (int)pow2_at_least((uint32_t)chunk_max);
-  const int acols = kAStages * Tr::kAcols;
-  a.nbuf = 2 * MT * a.acc_stride + acols <= 512 ? 2 : 1;
-  const int tcols = a.nbuf * MT * a.acc_stride + acols;
-  if (tcols > 512) return cudaErrorInvalidConfiguration;
-  a.tmem_cols = (int)pow2_at_least((uint32_t)tcols);
-  a.a_col0 = a.nbuf * MT * a.acc_stride;
+  a.a_stride = Tr::kAcols;
+  if (!Tr::kTmemA) {
+    a.nbuf = 2 * MT * a.acc_stride <= 512 ? 2 : 1;
+    a.tmem_cols = a.nbuf * MT * a.acc_stride;
+    a.a_col0 = 0;
+  } else if (2 * MT * a.acc_stride + kAStages * Tr::kAcols <= 512) {
+    a.nbuf = 2;
+    a.a_col0 = 2 * MT * a.acc_stride;
+    a.tmem_cols = (int)pow2_at_least((uint32_t)(a.a_col0 + kAStages * Tr::kAcols));
+  } else if (MT == 2 && kAStages == 2 && chunk_max <= 192) {
+    a.nbuf = 1;
+    a.acc_stride = 256;
+    a.a_col0 = 192;
+    a.a_stride = 256;
+    a.tmem_cols = 512;
+  } else {
+    return cudaErrorInvalidConfiguration;
+  }
+  if (a.tmem_cols > 512) return cudaErrorInvalidConfiguration;
   const int fixed = 1024 + kBarrierBytes + Tr::kXchg + Tr::kARing;
   const int avail = kSmemLimit - fixed;
   if (Tr::kQuant) {
@@ -864,11 +887,19 @@ cudaError_t launch_gemm(const Maps& m, GemmArgs a, int chunk_max, int num_sms, c
   return launch_k(kern, dim3(num_sms), dim3(Tr::kThreads), smem, s, m.w0, m.w1, m.b, m.w0d, m.w1d, m.bd, a);
 }
 
-// Quantised weights widen into TMEM when the accumulators leave room for the
-// widened A stages (chunks of at most 128 tokens); otherwise into shared memory.
+// Quantised weights widen into TMEM when two accumulator sets and the widened A
+// stages fit in its 512 columns (chunks of at most 64 tokens: decode-sized
+// batches, where it measured up to 11% faster for int4 and even for int8), and
+// for gate/up with chunks of at most 192 tokens in the interleaved layout (one
+// accumulator set: measured 8% faster on the int4 workload's 64-token experts).
+// Otherwise -- the down projection beyond 64 tokens, and 256-token chunks -- A
+// goes to shared memory, which keeps two accumulator sets where they fit: with
+// A in TMEM the 256-token int8 prefill measured 4-11% slower at 192-token chunks.
 template <int MODE, int WF, int MT>
 cudaError_t launch_quant(const Maps& m, const GemmArgs& a, int chunk_max, int num_sms, cudaStream_t s) {
-  if (chunk_max <= 128) return launch_gemm<MODE, WF, MT, 1>(m, a, chunk_max, num_sms, s);
+  const int acc = (int)pow2_at_least((uint32_t)chunk_max);  // TMEM columns of one tile's accumulator
+  if (2 * MT * acc + kAStages * MT * (kBK / 2) <= 512 || (MODE == 0 && MT == 2 && chunk_max <= 192))
+    return launch_gemm<MODE, WF, MT, 1>(m, a, chunk_max, num_sms, s);
   return launch_gemm<MODE, WF, MT, 0>(m, a, chunk_max, num_sms, s);
 }
 

@@ -56,6 +56,8 @@ inline int chunk_tokens(int T, int k, int E) {
   if (t > 128 && (long long)T * k <= 96LL * E) t = 128;
   return t;
 }
+// the token chunk of a layer's grouped GEMMs
+inline int gemm_chunk(const moe_desc& d, int T) { return chunk_tokens(T, d.k, d.E); }
 
 // Split of the router's reduction over H into S partial sums (summed in a
 // fixed order by the top-k kernel).  Depends on T only, so a masked layer and

@@ -193,14 +193,22 @@ static moe_status validate_T(int32_t T, int k) {
 // The tensor-core path needs bf16 activations, non-fp32 weights and 128-row tiles.
 static bool gemm_capable(const moe_desc& d) { return gemm_tc_supported(d); }
 
-// The tensor-core path streams weights with TMA and serves decode as well as
-// prefill; the SIMT GEMV path remains for fp32 layers and shapes the tensor
-// cores cannot tile.
+// The path by tokens per expert.  The tensor-core GEMM streams the weights with
+// TMA and serves decode as well as prefill; the SIMT weight-streaming GEMV serves
+// fp32 layers, shapes the tensor cores cannot tile, and the smallest int4 batches:
+// with at most one (token, slot) pair per kGemvPairsPerExpertInt4 experts on
+// average the GEMV widens only the rows it multiplies (and no token tiles),
+// which measured faster than the GEMM's full-tile dequantisation (1-4 tokens at
+// the Qwen3-30B-A3B widths).  bf16 and int8 weights take the GEMM at every batch
+// size: it measured at least as fast from one token up.
+constexpr int kGemvPairsPerExpertInt4 = 4;  // GEMV while T * k * 4 <= E
 static int choose_path(const moe_desc& d, int32_t T) {
-  (void)T;
   if (d.path == MOE_PATH_GEMV) return MOE_PATH_GEMV;
   if (d.path == MOE_PATH_GEMM) return MOE_PATH_GEMM;
-  return gemm_capable(d) ? MOE_PATH_GEMM : MOE_PATH_GEMV;
+  if (!gemm_capable(d)) return MOE_PATH_GEMV;
+  const bool int4 = d.wfmt == MOE_W_INT4_B32 || d.wfmt == MOE_W_INT4_B128;
+  if (int4 && (int64_t)T * d.k * kGemvPairsPerExpertInt4 <= d.E) return MOE_PATH_GEMV;
+  return MOE_PATH_GEMM;
 }
 
 // ------------------------------------------------------------------ workspace
@@ -363,18 +371,18 @@ static moe_status run_routed(const moe_desc* d, const void* x, int32_t T, const 
     // the plan was built together with the routing
   } else if (small_sort_ok(P, d->E)) {
     MOE_LAUNCH("small_sort", stream,
-               launch_small_sort(topk_idx, P, d->E, chunk_tokens(T, d->k, d->E), ws.counts, ws.offsets, ws.touched,
+               launch_small_sort(topk_idx, P, d->E, gemm_chunk(*d, T), ws.counts, ws.offsets, ws.touched,
                                  ws.group_base, ws.tile_base, ws.meta, ws.sorted_pair, dev->flags, stream));
   } else {
     MOE_LAUNCH("pair_histogram", stream, launch_pair_histogram(topk_idx, P, d->E, ws.chunk_hist, dev->flags, stream));
     MOE_LAUNCH("expert_scan", stream,
                launch_expert_scan(NC, d->E, ws.chunk_hist, ws.counts, ws.offsets, ws.touched, ws.group_base,
-                                  ws.tile_base, chunk_tokens(T, d->k, d->E), ws.meta, stream));
+                                  ws.tile_base, gemm_chunk(*d, T), ws.meta, stream));
     MOE_LAUNCH("pair_scatter", stream, launch_pair_scatter(topk_idx, P, d->E, ws.chunk_hist, ws.sorted_pair, stream));
   }
   if (path == MOE_PATH_GEMM) {
     MOE_LAUNCH("gather_rows", stream, launch_gather_rows(*d, x, ws, P, dev->num_sms, stream));
-    const int chunk = chunk_tokens(T, d->k, d->E);
+    const int chunk = gemm_chunk(*d, T);
     MOE_LAUNCH("gemm_gateup", stream,
                launch_gemm_gateup(*d, ws, P, chunk, dev->num_sms, dev->flags, stream, dense_up));
     MOE_LAUNCH("gemm_down", stream,
@@ -451,7 +459,7 @@ extern "C" moe_status moe_layer_forward(const moe_desc* d, const void* x, int32_
   MOE_LAUNCH("router_decode_logits", stream,
              launch_decode_logits(*d, x, T, ws.logits, S, dev->flags, stream, ws.meta + kMetaTopkDone));
   MOE_LAUNCH("router_topk_sort", stream,
-             launch_topk_sort(*d, ws.logits, S, T, topk_idx, topk_w, chunk_tokens(T, d->k, d->E), ws, dev->flags,
+             launch_topk_sort(*d, ws.logits, S, T, topk_idx, topk_w, gemm_chunk(*d, T), ws, dev->flags,
                               stream));
   if ((st = run_routed(d, x, T, topk_idx, topk_w, ws, path, dev, stream, true)) != MOE_OK) return st;
   MOE_LAUNCH("combine", stream, launch_combine(*d, topk_idx, T, ws.yp, yp_bf16(*d, T, path), y, stream));
@@ -549,7 +557,7 @@ extern "C" moe_status moe_forward_block(const moe_desc* d, const moe_shared_expe
   if (shared && path == MOE_PATH_GEMM && spath == MOE_PATH_GEMM && sd.wfmt == d->wfmt) {
     // the shared expert's units ride in the routed experts' grouped-GEMM launches
     const Workspace ss = carve_workspace(sd, T, static_cast<char*>(workspace) + shared_off);
-    const int chunk = chunk_tokens(T, sd.k, sd.E);
+    const int chunk = gemm_chunk(sd, T);
     const DenseGemm up{&sd, x, ss.hbuf, T, chunk};
     const DenseGemm down{&sd, ss.hbuf, ss.yp, T, chunk};
     if ((st = run_routed(d, x, T, topk_idx, topk_w, ws, path, dev, stream, false, &up, &down)) != MOE_OK) return st;
@@ -561,7 +569,7 @@ extern "C" moe_status moe_forward_block(const moe_desc* d, const moe_shared_expe
   if (shared) {
     Workspace ss = carve_workspace(sd, T, static_cast<char*>(workspace) + shared_off);
     float* ones = reinterpret_cast<float*>(static_cast<char*>(workspace) + ones_off);
-    const int chunk = chunk_tokens(T, 1, 1);
+    const int chunk = gemm_chunk(sd, T);
     MOE_LAUNCH("shared_plan", stream,
                launch_dense_plan(T, chunk, ss.counts, ss.offsets, ss.touched, ss.group_base, ss.tile_base, ss.meta,
                                  ss.sorted_pair, ones, stream));

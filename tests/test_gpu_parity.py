@@ -258,3 +258,22 @@ def test_stage_timing_reports_every_kernel(cid, T):
         moe.moe_stage_timing(False)
         moe.moe_stage_timing_only(None)
     assert set(only) == {"combine"} and only["combine"][0] == 2 and only["combine"][1] > 0
+
+
+@pytest.mark.parametrize("cid,T,kernel", [(4, 4, "gemv_gateup"), (4, 5, "gemm_gateup"), (4, 64, "gemm_gateup"),
+                                          (2, 1, "gemm_gateup"), (3, 1, "gemm_gateup")])
+def test_auto_path_by_tokens_per_expert(cid, T, kernel):
+    """The automatic path: int4 batches with at most one (token, slot) pair per four
+    experts on average take the weight-streaming GEMV, everything else the
+    tensor-core GEMM (the measured crossover); both give the oracle's result."""
+    prob = synth.make_problem(cid, T=T, H=256, E=128, I=128)
+    layer = layer_from_problem(prob)
+    x = x_to_device(prob)
+    moe.moe_stage_timing(True)
+    try:
+        y, idx, w = layer.layer(x)
+        times = moe.moe_stage_times()
+    finally:
+        moe.moe_stage_timing(False)
+    assert kernel in times
+    judge(prob, y, idx, w, logits=gpu_logits(layer, x))
