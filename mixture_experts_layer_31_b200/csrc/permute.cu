@@ -49,12 +49,18 @@ __global__ void __launch_bounds__(1024) expert_scan_kernel(int NC, int E, int32_
   pdl_trigger();
   __shared__ int warp_sums[32];
   const int e = threadIdx.x;
+  // two passes over the expert's column of chunk counts, each with kBatch loads in
+  // flight: the total first, then (once the expert's offset is known) the
+  // chunk bases, written in place
+  constexpr int kBatch = 16;
   int running = 0;
   if (e < E) {
-    for (int c = 0; c < NC; ++c) {
-      const int v = chunk_hist[(size_t)c * E + e];
-      chunk_hist[(size_t)c * E + e] = running;
-      running += v;
+    for (int c0 = 0; c0 < NC; c0 += kBatch) {
+      int v[kBatch];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) v[j] = c0 + j < NC ? chunk_hist[(size_t)(c0 + j) * E + e] : 0;
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) running += v[j];
     }
     counts[e] = running;
   }
@@ -62,7 +68,17 @@ __global__ void __launch_bounds__(1024) expert_scan_kernel(int NC, int E, int32_
   const int off = route_dev::block_exclusive_scan(e < E ? running : 0, warp_sums, &total);
   if (e < E) {
     offsets[e] = off;
-    for (int c = 0; c < NC; ++c) chunk_hist[(size_t)c * E + e] += off;
+    int base = off;
+    for (int c0 = 0; c0 < NC; c0 += kBatch) {
+      int v[kBatch];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) v[j] = c0 + j < NC ? chunk_hist[(size_t)(c0 + j) * E + e] : 0;
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        if (c0 + j < NC) chunk_hist[(size_t)(c0 + j) * E + e] = base;
+        base += v[j];
+      }
+    }
   }
   if (e == 0) offsets[E] = total;
   int ntouched;
@@ -83,6 +99,8 @@ __global__ void __launch_bounds__(1024) expert_scan_kernel(int NC, int E, int32_
     meta[1] = total;
     meta[2] = ngroups;
     meta[3] = nchunks;
+    meta[8] = 0;  // unit counters of the grouped GEMMs that follow
+    meta[9] = 0;
     group_base[ntouched] = ngroups;
     tile_base[ntouched] = nchunks;
   }
