@@ -370,7 +370,7 @@ def run_reference(args):
     return 0
 
 
-def roofline(prob, acc, kern, stages, path_used):
+def roofline(prob, acc, kern, stages, path_used, stock=True):
     """The dominant kernel's roofline: its algorithmic bytes and flops per launch over
     its average launch time inside the timed steps, bound by its arithmetic
     intensity against the measured ridge point; both fractions reported."""
@@ -392,7 +392,8 @@ def roofline(prob, acc, kern, stages, path_used):
                  "algorithmic_flops_per_launch": kflops, "traffic_overhead": acc["overhead"][kern],
                  "hbm_frac": hbm_frac, "tensor_frac": tc_frac,
                  "peak_source": "MEASURED_PEAKS.json hbm_gbs / bf16_tflops (burst), %s" % of})
-    roof["traffic"] = known_traffic(kern, prob.cfg["workload"])
+    # committed DRAM counts hold for the stock workload only (not a resized or block run)
+    roof["traffic"] = known_traffic(kern, prob.cfg["workload"]) if stock else None
     return roof
 
 
@@ -529,7 +530,8 @@ def measure(args, moe, prob, dev, local, world, headline: bool):
                                       "routing_counts": bool(stats),
                                       "block": ({"shared_I": prob.I_s, "residual": prob.residual is not None}
                                                 if block else None)}),
-        "roofline": roofline(prob, acc, kern, stages, path_used),
+        "roofline": roofline(prob, acc, kern, stages, path_used,
+                             stock=not (args.overrides or args.block) or not headline),
         "layer": {"algorithmic_bytes": acc["layer_bytes"], "algorithmic_flops": acc["layer_flops"],
                   "hbm_frac_of_step": acc["layer_bytes"] / (step_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                   "tensor_frac_of_step": acc["layer_flops"] / (step_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
