@@ -27,14 +27,17 @@
 //   warp 1          TMEM allocator; lane 0 issues tcgen05.mma, commits stages
 //   warp 2 lane 0   quantised weights only: TMA producer of the token boxes
 //   warps 4..11     epilogue (two 4-warp groups): tcgen05.ld -> activation / scales -> global
-//   warps 12..19    dequantisation (int8 / int4 only)
+//   warps 12..19    dequantisation (int8 / int4 only): one weight row per thread,
+//                   widened to bf16 into a shared-memory A ring or, where that
+//                   measured faster, into TMEM (the MMA then reads A from TMEM)
 // Quantised weights keep two rings so that a raw tile's slot is refilled as
 // soon as the dequant warps have widened it, not when the MMAs that use its
 // bf16 copy finish: the weight stream runs as many stages ahead as the raw
 // ring holds, while the token ring only needs to cover L2 latency.
-// TMEM holds two accumulator buffers when they fit (chunks up to 128 tokens),
-// so the epilogue of one unit overlaps the MMAs of the next.  Every wait is
-// bounded (MOE_FLAG_TIMEOUT).
+// TMEM holds two accumulator buffers when they fit (with A in shared memory:
+// chunks up to 128 tokens), so the epilogue of one unit overlaps the MMAs of the
+// next; launch_gemm lays out the accumulators and widened A stages.  Every wait
+// is bounded (MOE_FLAG_TIMEOUT).
 // A launch may carry a second, dense problem (the shared expert of the MoE
 // block: every token in order, weight 1, weights of its own) whose units follow
 // the routed ones, so both share the persistent grid.
