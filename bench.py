@@ -11,8 +11,11 @@ moe_forward_block or moe_expert_counts + moe_forward).  Default workload: the Ki
   value  tokens/s over the timed steps, inputs resident in HBM; each step timed
          with CUDA events on the launching stream, L2 flushed (a 512 MB write)
          between steps outside the timed intervals.
-  e2e    the same metric with x copied host->device from pinned memory and y
-         copied back inside each timed step.
+  e2e    the same metric with every step's x copied host->device from pinned memory
+         and its y copied back inside the timed region: pipelined as a serving loop
+         runs it (step i+1's input copy and step i-1's output copy overlap step i's
+         layer on streams of their own); the serial figure (copy in, layer, copy out,
+         one step after another) is reported beside it.
   roofline  the dominant kernel's algorithmic bytes (or flops) per launch over
          its average duration, from CUDA events around that kernel's launches
          inside the timed steps (the only kernel so bracketed there), against
@@ -483,34 +486,80 @@ def measure(args, moe, prob, dev, local, world, headline: bool):
     y_np = (y.view(torch.int16).cpu().numpy().view(np.uint16) if y.dtype == torch.bfloat16 else y.cpu().numpy())
     idx_np = idx.cpu().numpy()
 
-    # ---- end to end: pinned host x in, pinned host y out, copies inside each timed step
+    # ---- end to end: pinned host x in, pinned host y out, every step's copies inside
+    # the timed region.  Serial: copy in, layer, copy out, one step after another on the
+    # launching stream (L2 flushed between steps, outside the timed intervals).
+    # Pipelined (the reported e2e), as a serving loop runs it: the input copy of step
+    # i + 1 and the output copy of step i - 1 overlap the layer of step i on streams of
+    # their own, with double-buffered device x and y; one interval over all K steps, no
+    # flush (the expert weights are several times the L2).
     xh = x_host.pin_memory()
-    yh = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-    xd = torch.empty_like(x)
     rh = None if res_host is None else res_host.pin_memory()
-    rd = None if res is None else torch.empty_like(res)
+    yh = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for _ in range(2)]
+    xd = [torch.empty_like(x) for _ in range(2)]
+    yd = [torch.empty_like(y) for _ in range(2)]
+    rd = [None, None] if res is None else [torch.empty_like(res) for _ in range(2)]
     e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     for _ in range(2):
-        xd.copy_(xh, non_blocking=True)
-        if rd is not None:
-            rd.copy_(rh, non_blocking=True)
-        step(xd, y, rd)
-        yh.copy_(y, non_blocking=True)
+        xd[0].copy_(xh, non_blocking=True)
+        if rd[0] is not None:
+            rd[0].copy_(rh, non_blocking=True)
+        step(xd[0], yd[0], rd[0])
+        yh[0].copy_(yd[0], non_blocking=True)
     barrier()
     torch.cuda.synchronize(dev)
     for i in range(args.steps):
         flush.zero_()
         e_starts[i].record(stream)
-        xd.copy_(xh, non_blocking=True)
-        if rd is not None:
-            rd.copy_(rh, non_blocking=True)
-        step(xd, y, rd)
-        yh.copy_(y, non_blocking=True)
+        xd[0].copy_(xh, non_blocking=True)
+        if rd[0] is not None:
+            rd[0].copy_(rh, non_blocking=True)
+        step(xd[0], yd[0], rd[0])
+        yh[0].copy_(yd[0], non_blocking=True)
         e_ends[i].record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)) / args.steps, dev)
+    e2e_serial_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)) / args.steps, dev)
+
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def pipelined(n):
+        in_done = [torch.cuda.Event() for _ in range(n)]
+        comp_done = [torch.cuda.Event() for _ in range(n)]
+        out_done = [torch.cuda.Event() for _ in range(n)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        s_in.wait_event(t0)
+        for i in range(n):
+            bi = i & 1
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(comp_done[i - 2])  # step i - 2 has read this x buffer
+                xd[bi].copy_(xh, non_blocking=True)
+                if rd[bi] is not None:
+                    rd[bi].copy_(rh, non_blocking=True)
+                in_done[i].record(s_in)
+            stream.wait_event(in_done[i])
+            if i >= 2:
+                stream.wait_event(out_done[i - 2])  # this y buffer has been copied out
+            step(xd[bi], yd[bi], rd[bi])
+            comp_done[i].record(stream)
+            s_out.wait_event(comp_done[i])
+            with torch.cuda.stream(s_out):
+                yh[bi].copy_(yd[bi], non_blocking=True)
+                out_done[i].record(s_out)
+        stream.wait_event(out_done[n - 1])
+        t1.record(stream)
+        return t0, t1
+
+    pipelined(2)
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0, t1 = pipelined(args.steps)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, dev)
 
     # ---- per-kernel breakdown: a separate, untimed pass with every launch timed
     moe.moe_stage_timing(True)
@@ -540,11 +589,15 @@ def measure(args, moe, prob, dev, local, world, headline: bool):
         "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT,
                 "h2d_bytes_per_step": int(x.numel() * x.element_size())
                                       + (0 if res is None else int(res.numel() * res.element_size())),
-                "d2h_bytes_per_step": int(y.numel() * y.element_size())},
+                "d2h_bytes_per_step": int(y.numel() * y.element_size()),
+                "mode": "pipelined: step i+1's input copy and step i-1's output copy overlap step i's "
+                        "layer (double-buffered device x, y); one interval over the timed steps, no L2 flush",
+                "serial_value": world * T / (e2e_serial_ms * 1e-3),
+                "serial_mode": "copy in, layer, copy out per step on one stream, L2 flushed between steps"},
         "gpu_launches": int(launches),
         "clocks": clocks.summary(),
     }
-    del layer, x, y, idx, w, flush, xd, xh, yh
+    del layer, x, y, idx, w, flush, xd, yd, rd, xh, yh
     torch.cuda.synchronize(dev)
     torch.cuda.empty_cache()
     return fields, y_np, idx_np
